@@ -1,0 +1,15 @@
+"""fp64 CPU oracle (test infrastructure only).
+
+Plain numpy restatement of the Summaryformer frame memory and its attention,
+written from the model card "GTA world model: weights and inference code".
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
+leg use it; the CUDA library never imports it and it never imports the CUDA
+library.
+"""
+from .kvmemory import (Layout, FrameMemory, attend, attend_bits, attend_memory,
+                       softmax_weights, visible_history_mask, masked_history_attend,
+                       TINY, SERVED, SERVED_W16, SCALED)
+
+__all__ = ["Layout", "FrameMemory", "attend", "attend_bits", "attend_memory",
+           "softmax_weights", "visible_history_mask", "masked_history_attend",
+           "TINY", "SERVED", "SERVED_W16", "SCALED"]
