@@ -1,0 +1,143 @@
+/*
+ * wmkv.h -- Summaryformer frame memory and the attention that reads it, on B200 (sm_100a).
+ *
+ * Source of the method: the model card "GTA world model: weights and inference
+ * code" (lucidml/gta), sections "A frame is a record", "What a frame attends
+ * to" and "One buffer, no mask".
+ *
+ * Every block of the model keeps ONE preallocated key buffer and ONE value
+ * buffer, each laid out by rows as
+ *
+ *     | Z0: record(0) | RAW: (Y+1) rotating records | SUM: (W-Y) x X rotating summary rows |
+ *
+ * where a record is the frame's H*W raw tokens followed by its X summary
+ * tokens (R = H*W + X rows).  A row is `heads x d` bfloat16 values, row-major
+ * (token-major: element (row, h, c) sits at ((row*heads)+h)*d + c).
+ * Capacity C = R*(Y+2) + X*(W-Y) rows.  Slot conventions (they reproduce the
+ * page's served-shape example: frame 31 reuses frame 28's RAW slot, and frame
+ * 28's summary lands in the SUM slot that held frame 6's):
+ *   - frame 0 is written into Z0 and never evicted;
+ *   - frame t >= 1 is written into RAW slot (t-1) mod (Y+1);
+ *   - at the start of frame t >= Y+2, frame f = t-Y-1 leaves the raw window:
+ *     the K and V of its X summary rows are copied into SUM slot (f-1) mod (W-Y);
+ *   - attention reads buffer[0:end], the filled prefix, with no mask:
+ *     end(t) = R*(1 + min(t, Y+1)) + X*min(max(t-Y-1, 0), W-Y).
+ *
+ * Calls are asynchronous on the given CUDA stream (wm_stream_t is the same
+ * type as cudaStream_t; NULL is the legacy default stream).  Host-side
+ * checks run first: a call that fails them returns an error code and
+ * launches nothing.  Device pointers passed in (Q, K, V, O) are owned by the
+ * caller, must be 16-byte aligned, and must stay valid until the stream
+ * reaches the call; the library keeps no reference to them afterwards.
+ *
+ * A handle is used by one host thread at a time; the library holds no global
+ * mutable state.
+ */
+#ifndef WMKV_H
+#define WMKV_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define WM_API __attribute__((visibility("default")))
+#else
+#define WM_API
+#endif
+
+typedef struct CUstream_st* wm_stream_t;
+typedef struct wm_kvbuf wm_kvbuf;
+
+/* Error codes. */
+enum {
+  WM_OK = 0,
+  WM_ERR_INVALID_ARG = -1,  /* bad argument: range, NULL or misaligned pointer  */
+  WM_ERR_STATE = -2,        /* call out of order (see each call)                 */
+  WM_ERR_UNSUPPORTED = -3,  /* shape the kernels do not implement (d not 64/128) */
+  WM_ERR_OOM = -4,          /* device allocation failed                          */
+  WM_ERR_CUDA = -5,         /* a CUDA runtime call or launch failed              */
+  WM_ERR_TIMEOUT = -6       /* a kernel gave up a bounded wait (device flag)     */
+};
+
+/* Create the memory of one session: `blocks` per-block K/V buffer pairs on the
+ * current CUDA device, zero-filled, in one allocation of
+ * blocks * 2 * C * heads * d * 2 bytes (block b's K buffer first, then its V).
+ * Requirements: blocks >= 1, heads >= 1, d in {64, 128}, grid_h >= 1,
+ * grid_w >= 1, X >= 1, 0 <= Y <= W (W == Y gives an empty SUM region).
+ * Returns WM_ERR_INVALID_ARG / WM_ERR_UNSUPPORTED before touching the device,
+ * WM_ERR_OOM or WM_ERR_CUDA if allocation fails.  *out receives the handle. */
+WM_API int wm_kvbuf_create(wm_kvbuf** out, int blocks, int heads, int d, int grid_h, int grid_w, int X,
+                    int Y, int W);
+
+/* Free the buffers and the handle (synchronises the device first). */
+WM_API int wm_kvbuf_destroy(wm_kvbuf* h);
+
+/* Start frame t ("One buffer, no mask": when a frame falls out of the raw
+ * window its summary rows are copied RAW -> SUM).  t must be 0, then 1, 2, ...
+ * one call each, else WM_ERR_STATE.  For t >= Y+2 (and W > Y) one launch
+ * copies frame t-Y-1's X summary rows of K and of V into SUM, in every block. */
+WM_API int wm_advance(wm_kvbuf* h, int64_t t, wm_stream_t stream);
+
+/* Write frame t's record of `block` ("A frame is a record"): K and V are
+ * device arrays [R, heads, d] bf16 (raw rows first, then the X summary rows).
+ * t must equal the frame last passed to wm_advance (else WM_ERR_STATE).
+ * Frame 0 goes to Z0, frame t >= 1 to RAW slot (t-1) mod (Y+1).  May be called
+ * several times per frame (denoising passes, then the clean rewrite). */
+WM_API int wm_write_record(wm_kvbuf* h, int block, int64_t t, const void* K, const void* V,
+                    wm_stream_t stream);
+
+/* Dense unmasked attention of frame t's queries over buffer[0:end] of `block`:
+ *   O[i,h,:] = sum_j softmax_j(Q[i,h,:] . K[j,h,:] / sqrt(d)) V[j,h,:],  j < end.
+ * Q and O are device arrays [R, heads, d] bf16.  Scores, softmax and the
+ * accumulation are fp32 on the tensor cores (P rounded to bf16 for P.V); O is
+ * rounded to bf16.  Requires a wm_write_record(block, t) at the current t
+ * (else WM_ERR_STATE). */
+WM_API int wm_attend(wm_kvbuf* h, int block, const void* Q, void* O, wm_stream_t stream);
+
+/* Introspection (host only, no device work). */
+WM_API int64_t wm_end(const wm_kvbuf* h);                 /* end(t) at the current frame; -1 before t=0 */
+WM_API int64_t wm_capacity(const wm_kvbuf* h);            /* C */
+WM_API int64_t wm_current_frame(const wm_kvbuf* h);       /* last t passed to wm_advance, -1 before */
+WM_API int wm_raw_slot(const wm_kvbuf* h, int64_t t);     /* (t-1) mod (Y+1) for t >= 1; -1 for t < 1 */
+WM_API int wm_sum_slot(const wm_kvbuf* h, int64_t f);     /* (f-1) mod (W-Y) for f >= 1; -1 if none */
+/* Device pointers of block's K and V buffers, each [C, heads, d] bf16.  Owned
+ * by the handle; valid until wm_kvbuf_destroy. */
+WM_API int wm_kv_ptrs(const wm_kvbuf* h, int block, void** K, void** V);
+
+/* Synchronise the device, then read and clear the handle's device error flag:
+ * WM_ERR_TIMEOUT if a kernel gave up a bounded wait since the last call,
+ * WM_ERR_CUDA if the synchronisation itself failed, else WM_OK. */
+WM_API int wm_sync_status(wm_kvbuf* h);
+
+/* Static description of an error code. */
+WM_API const char* wm_strerror(int code);
+/* Text of the last CUDA error seen by this thread in a wm_* call ("" if none). */
+WM_API const char* wm_last_cuda_error(void);
+
+/* Pure layout arithmetic (no handle, no device) used by tests and tools. */
+WM_API int64_t wm_layout_capacity(int grid_h, int grid_w, int X, int Y, int W);
+WM_API int64_t wm_layout_end(int grid_h, int grid_w, int X, int Y, int W, int64_t t);
+WM_API int wm_layout_raw_slot(int Y, int64_t t);
+WM_API int wm_layout_sum_slot(int Y, int W, int64_t f);
+/* First row of frame t's record (Z0 for t = 0, its RAW slot otherwise). */
+WM_API int64_t wm_layout_record_row(int grid_h, int grid_w, int X, int Y, int64_t t);
+
+/* Dense attention with no frame memory.  The page contrasts the 6,528 keys
+ * of the served buffer with the 26,208 the same span would need at full
+ * resolution; this call runs that full-resolution comparison point:
+ *   O[i,h,:] = sum_j softmax_j(Q[i,h,:] . K[j,h,:] / sqrt(d)) V[j,h,:],  j < Lk,
+ * Q/O device [Lq, heads, d], K/V device [Lk, heads, d], all bf16, same
+ * kernel and numerics as wm_attend.  Lq >= 1, Lk >= 1, d in {64, 128}.
+ * `dev_status` is an optional device int (NULL to skip) that receives
+ * WM_ERR_TIMEOUT if the kernel gives up a bounded wait. */
+WM_API int wm_attend_dense(const void* Q, const void* K, const void* V, void* O, int64_t Lq, int64_t Lk,
+                    int heads, int d, int* dev_status, wm_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WMKV_H */

@@ -1,0 +1,116 @@
+// Record write and RAW -> SUM eviction: HBM-bound bit copies.
+//
+// Model card "GTA world model: weights and inference code", section "One
+// buffer, no mask": every pass stores the current frame's record in its slot;
+// a frame that drops out of the raw window keeps only its X summary rows (K
+// and V), moved from its RAW slot into SUM.  The page counts this small
+// per-block row copy as the whole price of long-term memory.
+//
+// Both are contiguous copies in the token-major buffer layout, moved as
+// 16-byte vectors with several independent loads in flight per thread and a
+// grid sized to the SM count.
+#include <cuda_runtime.h>
+
+#include "wmkv_internal.h"
+
+namespace wmkv {
+
+namespace {
+
+constexpr int COPY_THREADS = 256;
+constexpr int UNROLL = 4;
+
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ void copy_span(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                          int64_t n, int64_t first, int64_t stride) {
+  for (int64_t i = first; i < n; i += stride * UNROLL) {
+    uint4 r[UNROLL];
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      const int64_t idx = i + u * stride;
+      if (idx < n) r[u] = ld_stream(src + idx);
+    }
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      const int64_t idx = i + u * stride;
+      if (idx < n) dst[idx] = r[u];
+    }
+  }
+}
+
+// blockIdx.y selects array a (0) or b (1).
+__global__ void __launch_bounds__(COPY_THREADS) copy_pair_kernel(const uint4* __restrict__ a_src,
+                                                                 const uint4* __restrict__ b_src,
+                                                                 uint4* __restrict__ a_dst,
+                                                                 uint4* __restrict__ b_dst,
+                                                                 int64_t n) {
+  const uint4* src = blockIdx.y ? b_src : a_src;
+  uint4* dst = blockIdx.y ? b_dst : a_dst;
+  const int64_t stride = int64_t(gridDim.x) * COPY_THREADS;
+  copy_span(src, dst, n, int64_t(blockIdx.x) * COPY_THREADS + threadIdx.x, stride);
+}
+
+// blockIdx.y = 2*block + tensor (0 = K, 1 = V).
+__global__ void __launch_bounds__(COPY_THREADS) evict_kernel(uint8_t* base, int64_t block_stride,
+                                                             int64_t tensor_stride, int64_t src_off,
+                                                             int64_t dst_off, int64_t n) {
+  uint8_t* buf = base + int64_t(blockIdx.y >> 1) * block_stride + int64_t(blockIdx.y & 1) * tensor_stride;
+  const uint4* src = reinterpret_cast<const uint4*>(buf + src_off);
+  uint4* dst = reinterpret_cast<uint4*>(buf + dst_off);
+  const int64_t stride = int64_t(gridDim.x) * COPY_THREADS;
+  copy_span(src, dst, n, int64_t(blockIdx.x) * COPY_THREADS + threadIdx.x, stride);
+}
+
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+unsigned grid_x_for(int64_t n16, int parallel_arrays) {
+  // enough CTAs for every vector to be touched once with UNROLL in flight,
+  // capped at a few waves of the SM count across all arrays
+  const int64_t per_cta = int64_t(COPY_THREADS) * UNROLL;
+  int64_t want = (n16 + per_cta - 1) / per_cta;
+  const int64_t cap = (int64_t(sm_count()) * 8 + parallel_arrays - 1) / parallel_arrays;
+  if (want > cap) want = cap;
+  if (want < 1) want = 1;
+  return static_cast<unsigned>(want);
+}
+
+}  // namespace
+
+cudaError_t launch_copy_pair(const void* a_src, const void* b_src, void* a_dst, void* b_dst,
+                             int64_t n16, cudaStream_t stream) {
+  if (n16 <= 0) return cudaSuccess;
+  dim3 grid(grid_x_for(n16, 2), 2);
+  copy_pair_kernel<<<grid, COPY_THREADS, 0, stream>>>(
+      static_cast<const uint4*>(a_src), static_cast<const uint4*>(b_src), static_cast<uint4*>(a_dst),
+      static_cast<uint4*>(b_dst), n16);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_evict(void* base, int blocks, int64_t block_stride_bytes,
+                         int64_t tensor_stride_bytes, int64_t src_off_bytes, int64_t dst_off_bytes,
+                         int64_t n16, cudaStream_t stream) {
+  if (n16 <= 0 || blocks <= 0) return cudaSuccess;
+  dim3 grid(grid_x_for(n16, 2 * blocks), static_cast<unsigned>(2 * blocks));
+  evict_kernel<<<grid, COPY_THREADS, 0, stream>>>(static_cast<uint8_t*>(base), block_stride_bytes,
+                                                  tensor_stride_bytes, src_off_bytes, dst_off_bytes,
+                                                  n16);
+  return cudaGetLastError();
+}
+
+}  // namespace wmkv

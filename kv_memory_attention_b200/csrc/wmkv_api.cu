@@ -1,0 +1,278 @@
+// C ABI of the frame memory: the host state machine (slot arithmetic, the
+// filled prefix, call-order checks) and the launches behind it.
+//
+// Layout and rotation follow the model card "GTA world model: weights and
+// inference code": section "A frame is a record" (R = H*W raw + X summary
+// rows), "What a frame attends to" (Z0 whole, the last Y frames whole, older
+// in-window frames as summaries) and "One buffer, no mask" (one buffer per
+// block, | Z0 | RAW (Y+1) | SUM (W-Y) x X |, read = buffer[0:end], and the
+// worked example: frame 31 over frame 28's RAW slot, frame 28's summary over
+// frame 6's).  Frame t >= 1 uses RAW slot (t-1) mod (Y+1) and frame f's
+// summary SUM slot (f-1) mod (W-Y): with this base the filled rows stay a
+// contiguous prefix while the buffer fills.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/wmkv.h"
+#include "wmkv_internal.h"
+
+struct wm_kvbuf {
+  int device = 0;
+  int blocks = 0, heads = 0, d = 0, grid_h = 0, grid_w = 0, X = 0, Y = 0, W = 0;
+  int64_t HW = 0, R = 0, C = 0;
+  int64_t row_bytes = 0;     // heads * d * 2
+  int64_t tensor_bytes = 0;  // C * row_bytes (one K or V buffer)
+  int64_t block_bytes = 0;   // 2 * tensor_bytes
+  uint8_t* buf = nullptr;
+  int* status = nullptr;     // device error word
+  int64_t t = -1;            // current frame
+  std::vector<int64_t> written;  // per block: frame of the latest write_record
+};
+
+namespace {
+
+thread_local char g_last_cuda[256] = "";
+
+int cuda_fail(cudaError_t e) {
+  std::snprintf(g_last_cuda, sizeof(g_last_cuda), "%s: %s", cudaGetErrorName(e),
+                cudaGetErrorString(e));
+  return WM_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t capacity(int64_t hw, int64_t X, int64_t Y, int64_t W) {
+  return (hw + X) * (Y + 2) + X * (W - Y);
+}
+
+int64_t end_at(int64_t hw, int64_t X, int64_t Y, int64_t W, int64_t t) {
+  if (t < 0) return -1;
+  const int64_t R = hw + X;
+  const int64_t n_raw = t < Y + 1 ? t : Y + 1;
+  int64_t n_sum = t - Y - 1;
+  if (n_sum < 0) n_sum = 0;
+  if (n_sum > W - Y) n_sum = W - Y;
+  return R * (1 + n_raw) + X * n_sum;
+}
+
+int raw_slot(int64_t Y, int64_t t) { return t < 1 ? -1 : static_cast<int>((t - 1) % (Y + 1)); }
+
+int sum_slot(int64_t Y, int64_t W, int64_t f) {
+  return (f < 1 || W <= Y) ? -1 : static_cast<int>((f - 1) % (W - Y));
+}
+
+int64_t record_row(int64_t hw, int64_t X, int64_t Y, int64_t t) {
+  if (t < 0) return -1;
+  if (t == 0) return 0;
+  return (hw + X) * (1 + raw_slot(Y, t));
+}
+
+}  // namespace
+
+extern "C" {
+
+int wm_kvbuf_create(wm_kvbuf** out, int blocks, int heads, int d, int grid_h, int grid_w, int X,
+                    int Y, int W) {
+  if (!out) return WM_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (blocks < 1 || heads < 1 || heads > 65535 || grid_h < 1 || grid_w < 1 || X < 1 || Y < 0 ||
+      W < Y)
+    return WM_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return WM_ERR_UNSUPPORTED;
+  const int64_t hw = int64_t(grid_h) * grid_w;
+  const int64_t C = capacity(hw, X, Y, W);
+  const int64_t row_bytes = int64_t(heads) * d * 2;
+  // rows are addressed with 32-bit TMA coordinates
+  if (C >= (int64_t(1) << 31) || hw + X >= (int64_t(1) << 31)) return WM_ERR_INVALID_ARG;
+  const int64_t tensor_bytes = C * row_bytes;
+  if (tensor_bytes / row_bytes != C || tensor_bytes > (int64_t(1) << 46) / (2 * int64_t(blocks)))
+    return WM_ERR_INVALID_ARG;
+
+  wm_kvbuf* h = new (std::nothrow) wm_kvbuf;
+  if (!h) return WM_ERR_OOM;
+  h->blocks = blocks;
+  h->heads = heads;
+  h->d = d;
+  h->grid_h = grid_h;
+  h->grid_w = grid_w;
+  h->X = X;
+  h->Y = Y;
+  h->W = W;
+  h->HW = hw;
+  h->R = hw + X;
+  h->C = C;
+  h->row_bytes = row_bytes;
+  h->tensor_bytes = tensor_bytes;
+  h->block_bytes = 2 * tensor_bytes;
+  h->written.assign(blocks, -1);
+
+  cudaError_t e = cudaGetDevice(&h->device);
+  if (e != cudaSuccess) {
+    delete h;
+    return cuda_fail(e);
+  }
+  const size_t total = size_t(h->block_bytes) * size_t(blocks);
+  e = cudaMalloc(&h->buf, total);
+  if (e != cudaSuccess) {
+    delete h;
+    if (e == cudaErrorMemoryAllocation) {
+      cudaGetLastError();
+      return WM_ERR_OOM;
+    }
+    return cuda_fail(e);
+  }
+  e = cudaMalloc(&h->status, sizeof(int));
+  if (e == cudaSuccess) e = cudaMemset(h->buf, 0, total);
+  if (e == cudaSuccess) e = cudaMemset(h->status, 0, sizeof(int));
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    cudaFree(h->buf);
+    if (h->status) cudaFree(h->status);
+    delete h;
+    return cuda_fail(e);
+  }
+  *out = h;
+  return WM_OK;
+}
+
+int wm_kvbuf_destroy(wm_kvbuf* h) {
+  if (!h) return WM_ERR_INVALID_ARG;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaSetDevice(h->device);
+  cudaError_t e = cudaDeviceSynchronize();
+  cudaFree(h->buf);
+  cudaFree(h->status);
+  cudaSetDevice(dev);
+  delete h;
+  return e == cudaSuccess ? WM_OK : cuda_fail(e);
+}
+
+int wm_advance(wm_kvbuf* h, int64_t t, wm_stream_t stream) {
+  if (!h) return WM_ERR_INVALID_ARG;
+  if (t != h->t + 1) return WM_ERR_STATE;
+  const int64_t f = t - h->Y - 1;  // frame leaving the raw window
+  if (f >= 1 && h->W > h->Y) {
+    const int64_t src_row = h->R * (1 + raw_slot(h->Y, f)) + h->HW;
+    const int64_t dst_row = h->R * (h->Y + 2) + int64_t(h->X) * sum_slot(h->Y, h->W, f);
+    const int64_t n16 = int64_t(h->X) * h->row_bytes / 16;
+    cudaError_t e = wmkv::launch_evict(h->buf, h->blocks, h->block_bytes, h->tensor_bytes,
+                                       src_row * h->row_bytes, dst_row * h->row_bytes, n16,
+                                       reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  h->t = t;
+  return WM_OK;
+}
+
+int wm_write_record(wm_kvbuf* h, int block, int64_t t, const void* K, const void* V,
+                    wm_stream_t stream) {
+  if (!h || block < 0 || block >= h->blocks || !aligned16(K) || !aligned16(V))
+    return WM_ERR_INVALID_ARG;
+  if (h->t < 0 || t != h->t) return WM_ERR_STATE;
+  const int64_t row0 = record_row(h->HW, h->X, h->Y, t);
+  uint8_t* kdst = h->buf + int64_t(block) * h->block_bytes + row0 * h->row_bytes;
+  uint8_t* vdst = kdst + h->tensor_bytes;
+  const int64_t n16 = h->R * h->row_bytes / 16;
+  cudaError_t e = wmkv::launch_copy_pair(K, V, kdst, vdst, n16, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  h->written[block] = t;
+  return WM_OK;
+}
+
+int wm_attend(wm_kvbuf* h, int block, const void* Q, void* O, wm_stream_t stream) {
+  if (!h || block < 0 || block >= h->blocks || !aligned16(Q) || !aligned16(O))
+    return WM_ERR_INVALID_ARG;
+  if (h->t < 0 || h->written[block] != h->t) return WM_ERR_STATE;
+  const int64_t end = end_at(h->HW, h->X, h->Y, h->W, h->t);
+  const uint8_t* kbuf = h->buf + int64_t(block) * h->block_bytes;
+  const uint8_t* vbuf = kbuf + h->tensor_bytes;
+  cudaError_t e = wmkv::launch_attend(Q, kbuf, vbuf, O, h->R, end, h->heads, h->d, h->status,
+                                      reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return WM_OK;
+}
+
+int64_t wm_end(const wm_kvbuf* h) { return h ? end_at(h->HW, h->X, h->Y, h->W, h->t) : -1; }
+int64_t wm_capacity(const wm_kvbuf* h) { return h ? h->C : -1; }
+int64_t wm_current_frame(const wm_kvbuf* h) { return h ? h->t : -1; }
+int wm_raw_slot(const wm_kvbuf* h, int64_t t) { return h ? raw_slot(h->Y, t) : -1; }
+int wm_sum_slot(const wm_kvbuf* h, int64_t f) { return h ? sum_slot(h->Y, h->W, f) : -1; }
+
+int wm_kv_ptrs(const wm_kvbuf* h, int block, void** K, void** V) {
+  if (!h || block < 0 || block >= h->blocks || !K || !V) return WM_ERR_INVALID_ARG;
+  *K = h->buf + int64_t(block) * h->block_bytes;
+  *V = h->buf + int64_t(block) * h->block_bytes + h->tensor_bytes;
+  return WM_OK;
+}
+
+int wm_sync_status(wm_kvbuf* h) {
+  if (!h) return WM_ERR_INVALID_ARG;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e);
+  int flag = 0;
+  e = cudaMemcpy(&flag, h->status, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (flag != wmkv::DEV_OK) {
+    e = cudaMemset(h->status, 0, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e);
+    return WM_ERR_TIMEOUT;
+  }
+  return WM_OK;
+}
+
+const char* wm_strerror(int code) {
+  switch (code) {
+    case WM_OK: return "ok";
+    case WM_ERR_INVALID_ARG: return "invalid argument";
+    case WM_ERR_STATE: return "call out of order";
+    case WM_ERR_UNSUPPORTED: return "unsupported shape";
+    case WM_ERR_OOM: return "device allocation failed";
+    case WM_ERR_CUDA: return "CUDA error";
+    case WM_ERR_TIMEOUT: return "kernel gave up a bounded wait";
+    default: return "unknown error";
+  }
+}
+
+const char* wm_last_cuda_error(void) { return g_last_cuda; }
+
+int64_t wm_layout_capacity(int grid_h, int grid_w, int X, int Y, int W) {
+  if (grid_h < 1 || grid_w < 1 || X < 1 || Y < 0 || W < Y) return -1;
+  return capacity(int64_t(grid_h) * grid_w, X, Y, W);
+}
+
+int64_t wm_layout_end(int grid_h, int grid_w, int X, int Y, int W, int64_t t) {
+  if (grid_h < 1 || grid_w < 1 || X < 1 || Y < 0 || W < Y) return -1;
+  return end_at(int64_t(grid_h) * grid_w, X, Y, W, t);
+}
+
+int wm_layout_raw_slot(int Y, int64_t t) { return Y < 0 ? -1 : raw_slot(Y, t); }
+
+int wm_layout_sum_slot(int Y, int W, int64_t f) {
+  return (Y < 0 || W < Y) ? -1 : sum_slot(Y, W, f);
+}
+
+int64_t wm_layout_record_row(int grid_h, int grid_w, int X, int Y, int64_t t) {
+  if (grid_h < 1 || grid_w < 1 || X < 1 || Y < 0) return -1;
+  return record_row(int64_t(grid_h) * grid_w, X, Y, t);
+}
+
+int wm_attend_dense(const void* Q, const void* K, const void* V, void* O, int64_t Lq, int64_t Lk,
+                    int heads, int d, int* dev_status, wm_stream_t stream) {
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || Lq < 1 || Lk < 1 ||
+      heads < 1 || Lq >= (int64_t(1) << 31) || Lk >= (int64_t(1) << 31))
+    return WM_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return WM_ERR_UNSUPPORTED;
+  if ((Lq + 127) / 128 > 0x7FFFFFFF || heads > 65535) return WM_ERR_INVALID_ARG;
+  cudaError_t e = wmkv::launch_attend(Q, K, V, O, Lq, Lk, heads, d, dev_status,
+                                      reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return WM_OK;
+}
+
+}  // extern "C"

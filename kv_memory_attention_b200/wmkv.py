@@ -1,0 +1,249 @@
+"""ctypes binding of ``libwmkv.so`` (the C ABI declared in ``include/wmkv.h``).
+
+Argument marshalling only: every step of the frame memory and its attention
+runs in the library's CUDA kernels.  Tensors are passed as device pointers
+(``tensor.data_ptr()``); PyTorch is used by callers for device memory and
+streams.  There is no fallback: if the library is missing the import fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libwmkv.so")
+
+WM_OK = 0
+WM_ERR_INVALID_ARG = -1
+WM_ERR_STATE = -2
+WM_ERR_UNSUPPORTED = -3
+WM_ERR_OOM = -4
+WM_ERR_CUDA = -5
+WM_ERR_TIMEOUT = -6
+
+_c_int, _c_i64, _vp = ctypes.c_int, ctypes.c_int64, ctypes.c_void_p
+
+# name -> (restype, argtypes), in the order of include/wmkv.h
+SIGNATURES = {
+    "wm_kvbuf_create": (_c_int, [ctypes.POINTER(_vp), _c_int, _c_int, _c_int, _c_int, _c_int,
+                                 _c_int, _c_int, _c_int]),
+    "wm_kvbuf_destroy": (_c_int, [_vp]),
+    "wm_advance": (_c_int, [_vp, _c_i64, _vp]),
+    "wm_write_record": (_c_int, [_vp, _c_int, _c_i64, _vp, _vp, _vp]),
+    "wm_attend": (_c_int, [_vp, _c_int, _vp, _vp, _vp]),
+    "wm_end": (_c_i64, [_vp]),
+    "wm_capacity": (_c_i64, [_vp]),
+    "wm_current_frame": (_c_i64, [_vp]),
+    "wm_raw_slot": (_c_int, [_vp, _c_i64]),
+    "wm_sum_slot": (_c_int, [_vp, _c_i64]),
+    "wm_kv_ptrs": (_c_int, [_vp, _c_int, ctypes.POINTER(_vp), ctypes.POINTER(_vp)]),
+    "wm_sync_status": (_c_int, [_vp]),
+    "wm_strerror": (ctypes.c_char_p, [_c_int]),
+    "wm_last_cuda_error": (ctypes.c_char_p, []),
+    "wm_layout_capacity": (_c_i64, [_c_int, _c_int, _c_int, _c_int, _c_int]),
+    "wm_layout_end": (_c_i64, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_i64]),
+    "wm_layout_raw_slot": (_c_int, [_c_int, _c_i64]),
+    "wm_layout_sum_slot": (_c_int, [_c_int, _c_int, _c_i64]),
+    "wm_layout_record_row": (_c_i64, [_c_int, _c_int, _c_int, _c_int, _c_i64]),
+    "wm_attend_dense": (_c_int, [_vp, _vp, _vp, _vp, _c_i64, _c_i64, _c_int, _c_int, _vp, _vp]),
+}
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libwmkv.so not built at {LIB_PATH}; run python -m kv_memory_attention_b200.build")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+LIB = _load()
+
+
+class WmError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        msg = LIB.wm_strerror(code).decode()
+        if code == WM_ERR_CUDA:
+            msg += f" ({LIB.wm_last_cuda_error().decode()})"
+        super().__init__(f"{where}: {msg} [{code}]")
+        self.code = code
+
+
+def _check(code: int, where: str) -> int:
+    if code != WM_OK:
+        raise WmError(code, where)
+    return code
+
+
+def _ptr(x) -> int | None:
+    """Device pointer of a tensor, or an int address as is; None stays NULL."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(s) -> int | None:
+    """A torch.cuda.Stream, a raw cudaStream_t int, or None (torch's current stream)."""
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+# ---------------------------------------------------------------- ABI wrappers
+
+def wm_kvbuf_create(blocks: int, heads: int, d: int, grid_h: int, grid_w: int, X: int, Y: int,
+                    W: int) -> int:
+    h = _vp()
+    _check(LIB.wm_kvbuf_create(ctypes.byref(h), blocks, heads, d, grid_h, grid_w, X, Y, W),
+           "wm_kvbuf_create")
+    return h.value
+
+
+def wm_kvbuf_destroy(h: int) -> None:
+    _check(LIB.wm_kvbuf_destroy(h), "wm_kvbuf_destroy")
+
+
+def wm_advance(h: int, t: int, stream=None) -> None:
+    _check(LIB.wm_advance(h, t, _stream(stream)), "wm_advance")
+
+
+def wm_write_record(h: int, block: int, t: int, K, V, stream=None) -> None:
+    _check(LIB.wm_write_record(h, block, t, _ptr(K), _ptr(V), _stream(stream)), "wm_write_record")
+
+
+def wm_attend(h: int, block: int, Q, O, stream=None) -> None:
+    _check(LIB.wm_attend(h, block, _ptr(Q), _ptr(O), _stream(stream)), "wm_attend")
+
+
+def wm_end(h: int) -> int:
+    return LIB.wm_end(h)
+
+
+def wm_capacity(h: int) -> int:
+    return LIB.wm_capacity(h)
+
+
+def wm_current_frame(h: int) -> int:
+    return LIB.wm_current_frame(h)
+
+
+def wm_raw_slot(h: int, t: int) -> int:
+    return LIB.wm_raw_slot(h, t)
+
+
+def wm_sum_slot(h: int, f: int) -> int:
+    return LIB.wm_sum_slot(h, f)
+
+
+def wm_kv_ptrs(h: int, block: int) -> tuple[int, int]:
+    k, v = _vp(), _vp()
+    _check(LIB.wm_kv_ptrs(h, block, ctypes.byref(k), ctypes.byref(v)), "wm_kv_ptrs")
+    return k.value, v.value
+
+
+def wm_sync_status(h: int) -> None:
+    _check(LIB.wm_sync_status(h), "wm_sync_status")
+
+
+def wm_strerror(code: int) -> str:
+    return LIB.wm_strerror(code).decode()
+
+
+def wm_attend_dense(Q, K, V, O, Lq: int, Lk: int, heads: int, d: int, dev_status=None,
+                    stream=None) -> None:
+    _check(LIB.wm_attend_dense(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), Lq, Lk, heads, d,
+                               _ptr(dev_status), _stream(stream)), "wm_attend_dense")
+
+
+def wm_layout_capacity(grid_h, grid_w, X, Y, W) -> int:
+    return LIB.wm_layout_capacity(grid_h, grid_w, X, Y, W)
+
+
+def wm_layout_end(grid_h, grid_w, X, Y, W, t) -> int:
+    return LIB.wm_layout_end(grid_h, grid_w, X, Y, W, t)
+
+
+def wm_layout_raw_slot(Y, t) -> int:
+    return LIB.wm_layout_raw_slot(Y, t)
+
+
+def wm_layout_sum_slot(Y, W, f) -> int:
+    return LIB.wm_layout_sum_slot(Y, W, f)
+
+
+def wm_layout_record_row(grid_h, grid_w, X, Y, t) -> int:
+    return LIB.wm_layout_record_row(grid_h, grid_w, X, Y, t)
+
+
+# ---------------------------------------------------------------- convenience
+
+class KVMemory:
+    """One session's frame memory: owns a ``wm_kvbuf`` handle.
+
+    ``kv_views(block)`` returns torch views of the block's K and V buffers,
+    ``[C, heads, d]`` bf16 (read them only after the stream has reached the
+    calls that wrote them).
+    """
+
+    def __init__(self, blocks, heads, d, grid_h, grid_w, X, Y, W):
+        self.blocks, self.heads, self.d = blocks, heads, d
+        self.grid_h, self.grid_w, self.X, self.Y, self.W = grid_h, grid_w, X, Y, W
+        self.HW = grid_h * grid_w
+        self.R = self.HW + X
+        self.h = wm_kvbuf_create(blocks, heads, d, grid_h, grid_w, X, Y, W)
+        self.C = wm_capacity(self.h)
+
+    def close(self):
+        if self.h:
+            wm_kvbuf_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def advance(self, t, stream=None):
+        wm_advance(self.h, t, stream)
+
+    def write_record(self, block, t, K, V, stream=None):
+        wm_write_record(self.h, block, t, K, V, stream)
+
+    def attend(self, block, Q, O, stream=None):
+        wm_attend(self.h, block, Q, O, stream)
+
+    def end(self):
+        return wm_end(self.h)
+
+    def sync_status(self):
+        wm_sync_status(self.h)
+
+    def kv_views(self, block):
+        import torch
+        kp, vp = wm_kv_ptrs(self.h, block)
+        n = self.C * self.heads * self.d
+        return (_device_view(kp, n, torch.bfloat16).view(self.C, self.heads, self.d),
+                _device_view(vp, n, torch.bfloat16).view(self.C, self.heads, self.d))
+
+
+def _device_view(ptr: int, numel: int, dtype):
+    """A torch tensor aliasing library-owned device memory (no copy, no ownership)."""
+    import torch
+
+    class _Holder:
+        def __init__(self, p, nbytes):
+            self.__cuda_array_interface__ = {
+                "shape": (nbytes // 2,), "typestr": "<i2", "data": (p, False), "version": 3,
+                "strides": None}
+
+    t = torch.as_tensor(_Holder(ptr, numel * 2), device="cuda")
+    return t.view(dtype)

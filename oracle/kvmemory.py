@@ -19,12 +19,12 @@ What the page fixes, restated:
   * "One buffer, no mask": one preallocated K/V buffer per block with regions
     | Z0: record(0) | RAW: (Y+1) rotating records | SUM: (W-Y) x X rotating
     summary rows |; reading is buffer[0:end], the filled prefix, one dense
-    unmasked attention.  When a frame leaves the raw window the K and V of its
-    X summary tokens are copied RAW -> SUM and its raw rows are overwritten by
-    the next frame.  Worked example at the served shape: frame 31 is written
-    where frame 28 was, and frame 28's summary is written where frame 6's was.
-    Served numbers: 6,528 keys in the buffer versus 26,208 if the same span
-    were kept at full resolution.
+    unmasked attention.  A frame that drops out of the raw window keeps only
+    its X summary rows (K and V), moved from RAW into SUM; the next frame then
+    reuses its RAW slot.  Served-shape example: frame 31 takes frame 28's RAW
+    slot and frame 28's summary takes the SUM slot of frame 6's.  Served
+    numbers: 6,528 buffered keys, against 26,208 for the same span at full
+    resolution.
   * "The rest of the model", Sampling: each frame takes three denoising passes
     plus one clean pass that rewrites the frame's entry in memory.
 
@@ -146,6 +146,7 @@ class FrameMemory:
     """
     layout: Layout
     blocks: int
+    track_records: bool = True   # keep every record for check_against_records (small runs)
     t: int = -1
     K: np.ndarray = field(init=False)
     V: np.ndarray = field(init=False)
@@ -175,7 +176,8 @@ class FrameMemory:
         f = L.evicted_frame(t)
         if f is not None and L.W > L.Y:
             s = L.raw_slot(f)
-            assert self.raw_tag[s] == f
+            if self.raw_tag[s] != f:
+                raise ValueError(f"frame {f} leaves the raw window but was never written")
             r0, r1 = L.raw_rows(s)
             src0 = r0 + L.HW                       # summary tokens follow the raw ones
             u = L.sum_slot(f)
@@ -198,7 +200,8 @@ class FrameMemory:
         self.V[block, r0:r1] = v
         if t >= 1:
             self.raw_tag[L.raw_slot(t)] = t
-        self.records[(block, t)] = (k.copy(), v.copy())
+        if self.track_records:
+            self.records[(block, t)] = (k.copy(), v.copy())
         self.written.add(block)
 
     def prefix(self, block: int):
@@ -208,6 +211,7 @@ class FrameMemory:
 
     def check_against_records(self) -> None:
         """Every filled row equals the row it came from; unfilled rows are zero."""
+        assert self.track_records, "records are not kept for this memory"
         L = self.layout
         t = self.t
         for b in range(self.blocks):

@@ -18,6 +18,12 @@ Distributions (the workloads the model card describes carry K, V, Q rows of
   * Q, K, V: N(0, 1) float32, rounded to nearest-even bfloat16;
   * K row scale (batch-of-sessions workload): one U(0.5, 2) float32 per token
     row, shared by all heads and channels, applied in float32 before rounding.
+
+Record-sized tensors (``record_inputs``) are windows of one shared pool of
+2^25 N(0,1) float32 samples drawn once from Philox with the base seed; the
+window start is the tensor's 64-bit key modulo the pool size (wrapping
+around).  Each tensor is still N(0,1) and fixed by its tuple, and a
+28-block, 41-frame rollout needs seconds instead of minutes to generate.
 """
 from __future__ import annotations
 
@@ -57,13 +63,14 @@ def _gen(seed: int) -> np.random.Generator:
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     """Round float32 to bfloat16 (round to nearest, ties to even); returns uint16 bits.
 
-    Inputs are finite (normal samples), so NaN handling is not needed.
+    Inputs are finite and far below the float32 maximum (normal samples), so
+    the 32-bit sum below cannot carry out of the word and NaN handling is not
+    needed.
     """
     x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
-    lsb = (u >> np.uint64(16)) & np.uint64(1)
-    r = (u + np.uint64(0x7FFF) + lsb) >> np.uint64(16)
-    return r.astype(np.uint16)
+    u = x.view(np.uint32)
+    r = u + (np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1)))
+    return (r >> np.uint32(16)).astype(np.uint16)
 
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
@@ -98,6 +105,41 @@ def scaled_rows_bf16(seed: int, scale_seed: int, rows: int, heads: int, d: int,
     return f32_to_bf16_bits(z * s[:, None, None])
 
 
+POOL_LOG2 = 25
+_POOL = {}
+
+
+def _pool():
+    if "f32" not in _POOL:
+        z = _gen(splitmix64(BASE_SEED ^ 0x9001)).standard_normal(1 << POOL_LOG2, dtype=np.float32)
+        _POOL["f32"] = z
+        _POOL["bf16"] = f32_to_bf16_bits(z)
+    return _POOL
+
+
+def _window(arr: np.ndarray, seed: int, n: int) -> np.ndarray:
+    size = arr.shape[0]
+    assert n <= size
+    start = seed % size
+    if start + n <= size:
+        return arr[start:start + n].copy()
+    return np.concatenate([arr[start:], arr[:n - (size - start)]])
+
+
+def pool_normal_bf16(seed: int, shape) -> np.ndarray:
+    """N(0,1) bf16 bits of ``shape``: the pool window selected by ``seed``."""
+    n = int(np.prod(shape))
+    return _window(_pool()["bf16"], seed, n).reshape(shape)
+
+
+def pool_scaled_rows_bf16(seed: int, scale_seed: int, rows: int, heads: int, d: int,
+                          lo: float = 0.5, hi: float = 2.0) -> np.ndarray:
+    """Pool window as float32 rows, each times its own U(lo, hi), then rounded to bf16."""
+    z = _window(_pool()["f32"], seed, rows * heads * d).reshape(rows, heads, d)
+    s = uniform_f32(scale_seed, rows, lo, hi)
+    return f32_to_bf16_bits(z * s[:, None, None])
+
+
 def record_inputs(config: int, session: int, block: int, frame: int, step: int,
                   rows: int, heads: int, d: int, k_row_scale: bool = False):
     """(Q, K, V) bf16 bit arrays ``[rows, heads, d]`` for one write+attend step."""
@@ -105,11 +147,11 @@ def record_inputs(config: int, session: int, block: int, frame: int, step: int,
     sq = seed_for(config, session, block, frame, step, T_Q)
     sk = seed_for(config, session, block, frame, step, T_K)
     sv = seed_for(config, session, block, frame, step, T_V)
-    q = normal_bf16(sq, shape)
+    q = pool_normal_bf16(sq, shape)
     if k_row_scale:
         ss = seed_for(config, session, block, frame, step, T_KSCALE)
-        k = scaled_rows_bf16(sk, ss, rows, heads, d)
+        k = pool_scaled_rows_bf16(sk, ss, rows, heads, d)
     else:
-        k = normal_bf16(sk, shape)
-    v = normal_bf16(sv, shape)
+        k = pool_normal_bf16(sk, shape)
+    v = pool_normal_bf16(sv, shape)
     return q, k, v
