@@ -1,0 +1,482 @@
+"""Benchmark: steady-state frame-steps of the Summaryformer frame memory on B200.
+
+One step (one "frame") = wm_advance(t) (RAW -> SUM eviction in all 28 blocks)
+followed, for each of the 28 blocks, by wm_write_record (the frame's K/V
+record) and wm_attend (1104 queries x 6,528 keys x 16 heads x 64), at the
+served shape 24x42 + X=96, Y=2, W=24, in steady state (t >= 31).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line on rank 0.  ``value`` = frame-steps/s over all ranks
+(each rank runs its own independent session: weak scaling, no collective on
+the data path), timed with CUDA events between a barrier + synchronize on
+both sides, max over ranks.  ``--impl reference`` times the fp64 CPU oracle on
+the host cores instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import seeded_inputs as si  # noqa: E402
+
+METRIC = "steady-state frames/s (28 blocks attend+evict, 6528 keys); % bf16 TC peak"
+UNIT = "frames/s"
+
+# served shape (model card: 24x42 latent grid, X=96, Y=2, W=24 trained window,
+# 28 blocks, heads of 64; the synthetic workload uses 16 heads)
+BLOCKS, HEADS, D, GH, GW, X, Y, W = 28, 16, 64, 24, 42, 96, 2, 24
+HW = GH * GW
+R = HW + X
+C = R * (Y + 2) + X * (W - Y)
+T_STEADY = 31
+ATTN_FLOP = 4 * R * C * D * HEADS                 # QK^T + PV, multiply-add = 2
+EVICT_BYTES = 2 * 2 * X * HEADS * D * 2 * BLOCKS  # read + write, K and V, all blocks
+WRITE_BYTES = 2 * 2 * R * HEADS * D * 2           # read + write, K and V, one block
+WORKLOAD = (f"served frame-step: advance (evict) + {BLOCKS} x (write_record + attend), "
+            f"grid {GH}x{GW} + X={X}, Y={Y}, W={W}, {HEADS} heads x {D}, "
+            f"{R} queries x {C} keys, steady state t>={T_STEADY}, one session per GPU")
+CONFIG_ID = 3
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p["bf16_tflops_sustained"], p["bf16_tflops"], p["hbm_gbs"], "measured"
+    except Exception:
+        return 1400.0, 1590.0, 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", str(self.gpu_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- distributed
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_pg(world, backend):
+    import datetime
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args, world, rank, local):
+    import torch
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_pg(world, "nccl")
+    import kv_memory_attention_b200 as wm
+
+    kv = wm.KVMemory(BLOCKS, HEADS, D, GH, GW, X, Y, W)
+    pool = torch.from_numpy(si._pool()["bf16"].view(np.int16)).to(device).view(torch.bfloat16)
+    psize = pool.shape[0]
+    n = R * HEADS * D
+
+    def window(seed):
+        s = seed % psize
+        if s + n <= psize:
+            return pool[s:s + n].view(R, HEADS, D).clone()
+        return torch.cat([pool[s:], pool[:n - (psize - s)]]).view(R, HEADS, D)
+
+    # distinct per-block inputs (28 x Q, K, V = 190 MB resident in HBM)
+    Q = [window(si.seed_for(CONFIG_ID, rank, b, 0, 0, si.T_Q)) for b in range(BLOCKS)]
+    K = [window(si.seed_for(CONFIG_ID, rank, b, 0, 0, si.T_K)) for b in range(BLOCKS)]
+    V = [window(si.seed_for(CONFIG_ID, rank, b, 0, 0, si.T_V)) for b in range(BLOCKS)]
+    O = [torch.empty(R, HEADS, D, dtype=torch.bfloat16, device=device) for _ in range(BLOCKS)]
+    stream = torch.cuda.current_stream()
+
+    # fill the memory up to steady state
+    t = 0
+    for t in range(T_STEADY):
+        kv.advance(t)
+        for b in range(BLOCKS):
+            kv.write_record(b, t, K[b], V[b])
+    t = T_STEADY
+
+    def step(t, ev=None):
+        kv.advance(t, stream)
+        for b in range(BLOCKS):
+            kv.write_record(b, t, K[b], V[b], stream)
+            if ev is not None:
+                ev[b][0].record(stream)
+            kv.attend(b, Q[b], O[b], stream)
+            if ev is not None:
+                ev[b][1].record(stream)
+
+    for _ in range(args.warmup):
+        step(t)
+        t += 1
+    torch.cuda.synchronize()
+    kv.sync_status()
+
+    # ------------------------------------------------ timed region (device-resident inputs)
+    ev_attn = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(BLOCKS)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for s in range(args.steps):
+            step(t, ev_attn[s])
+            t += 1
+        stop.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    kv.sync_status()
+    elapsed_ms = max_over_ranks(start.elapsed_time(stop), world, device)
+    attn_ms = [a.elapsed_time(b) for row in ev_attn for (a, b) in row]
+    attn_avg_ms = statistics.mean(attn_ms)
+    launches = args.steps * (1 + 2 * BLOCKS)
+
+    # ------------------------------------------------ end to end: host buffers through the ABI
+    e2e = run_e2e(args, torch, wm, kv, t, rank, world, device, Q, K, V)
+    t = e2e.pop("_t")
+    kv.sync_status()
+
+    value = world * args.steps / (elapsed_ms / 1e3)
+    sustained, burst, hbm, src = peaks()
+    achieved_tflops = ATTN_FLOP / (attn_avg_ms * 1e-3) / 1e12
+    step_tflops = BLOCKS * ATTN_FLOP * args.steps / (elapsed_ms / 1e3) / 1e12
+    traffic = load_traffic()
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(elapsed_ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "blocks": BLOCKS, "heads": HEADS, "head_dim": D,
+                   "grid": f"{GH}x{GW}", "X": X, "Y": Y, "W": W, "queries": R, "keys": C,
+                   "parallelism": f"replicas x{world} (independent sessions)",
+                   "l2": "no flush: per step the 28 blocks touch 748 MB of K/V buffers + 190 MB of "
+                         "inputs, far above the 126 MB L2"},
+        "tflops_per_step": round(step_tflops, 1),
+        "frac_of_bf16_peak_step": round(step_tflops / sustained, 4),
+        "served_frames_per_s": round(value / 4, 3),
+        "roofline": {"kernel": "attend_kernel<64>", "bound": "tensor",
+                     "achieved": round(achieved_tflops, 1), "peak": sustained, "unit": "TFLOP/s",
+                     "frac": round(achieved_tflops / sustained, 4),
+                     "peak_source": f"bf16_tflops_sustained ({src})",
+                     "avg_launch_us": round(attn_avg_ms * 1e3, 2),
+                     "flop_per_launch": ATTN_FLOP, "traffic": traffic},
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    kv.close()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_e2e(args, torch, wm, kv, t, rank, world, device, Qd, Kd, Vd):
+    """Same steps with inputs in pinned host memory: H2D of Q/K/V and D2H of O every step."""
+    hq = [x.cpu().pin_memory() for x in Qd]
+    hk = [x.cpu().pin_memory() for x in Kd]
+    hv = [x.cpu().pin_memory() for x in Vd]
+    ho = [torch.empty(R, HEADS, D, dtype=torch.bfloat16).pin_memory() for _ in range(BLOCKS)]
+    dq = [torch.empty_like(x) for x in Qd]
+    dk = [torch.empty_like(x) for x in Kd]
+    dv = [torch.empty_like(x) for x in Vd]
+    do = [torch.empty(R, HEADS, D, dtype=torch.bfloat16, device=device) for _ in range(BLOCKS)]
+    comp = torch.cuda.current_stream()
+    s_in = torch.cuda.Stream()
+    s_out = torch.cuda.Stream()
+    used = [torch.cuda.Event() for _ in range(BLOCKS)]     # staging inputs consumed, O written
+    landed = [torch.cuda.Event() for _ in range(BLOCKS)]   # H2D of the block's inputs finished
+    copied = [torch.cuda.Event() for _ in range(BLOCKS)]   # D2H of the block's O finished
+    for b in range(BLOCKS):
+        used[b].record(comp)
+        copied[b].record(s_out)
+
+    def step(t):
+        for b in range(BLOCKS):
+            s_in.wait_event(used[b])
+            with torch.cuda.stream(s_in):
+                dq[b].copy_(hq[b], non_blocking=True)
+                dk[b].copy_(hk[b], non_blocking=True)
+                dv[b].copy_(hv[b], non_blocking=True)
+            landed[b].record(s_in)
+        wm.wm_advance(kv.h, t, comp)
+        for b in range(BLOCKS):
+            comp.wait_event(landed[b])
+            comp.wait_event(copied[b])
+            wm.wm_write_record(kv.h, b, t, dk[b], dv[b], comp)
+            wm.wm_attend(kv.h, b, dq[b], do[b], comp)
+            used[b].record(comp)
+            s_out.wait_event(used[b])
+            with torch.cuda.stream(s_out):
+                ho[b].copy_(do[b], non_blocking=True)
+            copied[b].record(s_out)
+
+    for _ in range(max(1, args.warmup)):
+        step(t)
+        t += 1
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    start.record(comp)
+    s_in.wait_event(start)
+    s_out.wait_event(start)
+    for _ in range(args.steps):
+        step(t)
+        t += 1
+    comp.wait_stream(s_out)
+    stop.record(comp)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(start.elapsed_time(stop), world, device)
+    nbytes = R * HEADS * D * 2
+    return {"value": round(world * args.steps / (ms / 1e3), 3), "unit": UNIT,
+            "h2d_bytes_per_step": 3 * BLOCKS * nbytes, "d2h_bytes_per_step": BLOCKS * nbytes,
+            "ms_per_step": round(ms / args.steps, 4),
+            "how": "pinned host Q/K/V copied in on a copy stream, O copied out on another, "
+                   "overlapped with the kernels block by block", "_t": t}
+
+
+TRAFFIC_SUMMARY = os.path.join(ROOT, "profiles", "attend_kernel_served.md")
+ATTEND_SOURCE = os.path.join(ROOT, "kv_memory_attention_b200", "csrc", "attend_sm100.cu")
+
+
+def source_digest() -> str:
+    import hashlib
+    with open(ATTEND_SOURCE, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def load_traffic():
+    """DRAM bytes per attend launch from the committed ncu summary.
+
+    The summary records the sha256 prefix of the kernel source it was taken
+    from (``source_sha256: ...``) and ``dram_bytes_per_launch: N``; if the
+    source has changed since, the figure is stale and null is reported.
+    """
+    try:
+        fields = {}
+        with open(TRAFFIC_SUMMARY) as f:
+            for ln in f:
+                if ":" in ln:
+                    k, v = ln.split(":", 1)
+                    fields[k.strip().strip("-* `")] = v.strip().strip("`")
+        if fields.get("source_sha256") != source_digest():
+            return None
+        return int(float(fields["dram_bytes_per_launch"]))
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def _oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        if info:
+            return max(i.get("num_threads", 1) for i in info)
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+class OracleStepper:
+    """The fp64 oracle stepping one served block through steady-state frames.
+
+    Each ``step(budget)`` advances the oracle's memory one frame (eviction),
+    writes the block's record and runs attention for query rows (all 16
+    heads, 6,528 keys) until ``budget`` seconds of attention have been spent;
+    the time is extrapolated to a full frame-step of 28 blocks x 1104 rows.
+    """
+
+    def __init__(self):
+        from oracle import FrameMemory, Layout
+        self.L = Layout(GH, GW, X, Y, W, heads=HEADS, d=D)
+        self.mem = FrameMemory(self.L, 1, track_records=False)
+        for t in range(T_STEADY):
+            self.mem.advance(t)
+            _, k, v = si.record_inputs(CONFIG_ID, 0, 0, t, 0, R, HEADS, D)
+            self.mem.write_record(0, t, k, v)
+        self.t = T_STEADY
+        self.next_row = 0
+
+    def step(self, budget_s: float):
+        from oracle import attend_memory
+        q, k, v = si.record_inputs(CONFIG_ID, 0, 0, self.t, 0, R, HEADS, D)
+        t0 = time.perf_counter()
+        self.mem.advance(self.t)
+        t_evict = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        self.mem.write_record(0, self.t, k, v)
+        t_write = time.perf_counter() - t0
+        rows_done, t_attn = 0, 0.0
+        while True:
+            rows = (np.arange(self.next_row, self.next_row + 128)) % R
+            self.next_row = (self.next_row + 128) % R
+            t0 = time.perf_counter()
+            attend_memory(self.mem, 0, q, rows=rows)
+            t_attn += time.perf_counter() - t0
+            rows_done += 128
+            if t_attn >= budget_s:
+                break
+        self.t += 1
+        per_step = BLOCKS * (R * t_attn / rows_done + t_write) + t_evict
+        return per_step, rows_done, t_attn
+
+
+def cpu_baseline(budget_s: float):
+    per_step, rows, t_attn = OracleStepper().step(budget_s)
+    return {"value": round(1.0 / per_step, 6), "unit": UNIT, "cores": _oracle_threads(),
+            "kind": "oracle",
+            "sample": f"{rows} query rows x 16 heads x 6528 keys of one block ({t_attn:.1f} s fp64 numpy), "
+                      f"plus one eviction and one record write of that block's memory, "
+                      f"extrapolated to 28 blocks x 1104 rows",
+            "host_cpus": len(os.sched_getaffinity(0))}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    # size each step so the whole run stays within ~2 minutes
+    n_steps = args.warmup + args.steps
+    budget = max(0.05, min(2.0, 120.0 / max(1, n_steps)))
+    stepper = OracleStepper()
+    for _ in range(args.warmup):
+        stepper.step(budget)
+    per = []
+    rows_total, attn_total = 0, 0.0
+    for _ in range(args.steps):
+        s, rows, ta = stepper.step(budget)
+        per.append(s)
+        rows_total += rows
+        attn_total += ta
+    total = sum(per)
+    value = args.steps / total
+    cores = _oracle_threads()
+    line = {"metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD, "blocks": BLOCKS, "heads": HEADS, "head_dim": D,
+                       "grid": f"{GH}x{GW}", "X": X, "Y": Y, "W": W, "queries": R, "keys": C,
+                       "parallelism": "host cores (fp64 oracle)"},
+            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"per step about {budget:.2f} s of query rows of one block "
+                                       f"({rows_total} rows in all) plus one eviction and one record "
+                                       f"write, extrapolated to a full 28-block frame-step"},
+            "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)      # at least 3 untimed warm-up steps
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()
