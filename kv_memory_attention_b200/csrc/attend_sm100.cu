@@ -5,23 +5,40 @@
 // block, no mask): for every head h and query row i
 //     O[i,h,:] = sum_{j<lk} softmax_j(Q[i,h,:] . K[j,h,:] / sqrt(d)) V[j,h,:]
 //
-// Design (one CTA per 128-query tile and head):
+// Design (one CTA per 128-query tile and head, 384 threads = 3 warpgroups):
 //   warp 8      TMA producer: Q tile once, then K_j / V_j tiles (128 keys) into
-//               an NS-stage ring, 128-byte swizzled, zero-filled past lk.
-//   warp 9      owns TMEM (512 columns) and issues every tcgen05.mma:
-//                 S_j = Q K_j^T          (SS: both operands K-major in smem)
-//                 O_g += P_j V_j         (TS: P from TMEM, V MN-major in smem)
-//   warps 0-3   softmax warpgroup 0: even KV tiles, S0/O0 in TMEM
-//   warps 4-7   softmax warpgroup 1: odd KV tiles, S1/O1 in TMEM
-// Each softmax thread owns one query row (= one TMEM lane).  It reads its S
-// row, updates the running max m and sum l (exp2 with log2(e)/sqrt(d)
-// folded into the score scale), rescales its O row in TMEM when m grew,
-// writes P as bf16 over the first half of its S columns, and signals the MMA
-// warp.  The two warpgroups ping-pong so that the tensor core computes one
-// tile's S while the other tile's softmax runs.  At the end the two partial
-// results (m0,l0,O0) and (m1,l1,O1) are merged row by row and stored as bf16.
+//               separate K and V rings (K two tiles ahead), 128-byte swizzled,
+//               zero-filled past lk.
+//   warp 9      owns TMEM (512 columns) and issues S_j = Q K_j^T
+//               (tcgen05.mma SS: both operands K-major in smem)
+//   warp 10     issues O_g += P_j V_j (tcgen05.mma TS: P from TMEM, V MN-major
+//               in smem); two issuing threads keep the tensor core fed while
+//               each waits on barriers and commits.  For d = 128 warp 9
+//               issues both, in order.
+//   warps 0-3   softmax warpgroup 0: even key tiles, S0/P0/O0 in TMEM
+//   warps 4-7   softmax warpgroup 1: odd key tiles, S1/P1/O1 in TMEM
+//   warp 11     idle (it completes the control warpgroup 8-11)
+// The control warpgroup gives registers back (setmaxnreg) so that each
+// softmax thread can hold its 128 scores without spilling.  Each softmax
+// thread owns one query row (= one TMEM lane).
 //
-// Every mbarrier wait is bounded (2 s); a CTA that gives up sets a shared
+// Pipeline per warpgroup g and its tile j (= g, g+2, ...):
+//   wait S_full[g] -> load the S row into registers -> arrive S_free[g]
+//   (for d = 64, P has its own TMEM columns, so the MMA warp can already issue
+//   S_{j+2} into S_g while this tile's softmax runs) -> row max; the exponent
+//   reference m moves only when the max grows by more than 2^8 (the final
+//   division by l is exact either way) -> p = 2^(s*log2(e)/sqrt(d) - m) in
+//   registers (MUFU, optionally part on the FMA pipe) -> wait O_done[g] (P.V
+//   of tile j-2 finished: O_g is stable and P_g is free; waiting only now
+//   hides the MMA round trip behind the exponentials) -> rescale O_g if m
+//   moved -> P as bf16 into TMEM -> arrive P_full[g].
+// For d = 128 the TMEM budget (2 S + 2 O of 128 columns) leaves no room for a
+// separate P, so P overwrites the first half of S and S_{j+2} is issued only
+// after P_j.V_j has completed (O_done).
+// The two warpgroups' partial results (m, l, O) are merged row by row at the
+// end and stored as bf16.
+//
+// Every mbarrier wait is bounded (about 2 s); a CTA that gives up sets a shared
 // abort flag, records DEV_TIMEOUT in the caller's status word, drains what it
 // issued, frees TMEM and exits.
 #include <cuda.h>
@@ -40,42 +57,86 @@ namespace {
 
 constexpr int BM = 128;  // queries per tile
 constexpr int BN = 128;  // keys per KV tile
-constexpr int NUM_THREADS = 320;
-constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
-constexpr uint64_t DRAIN_LIMIT_NS = 200000000ull;
+constexpr int NUM_THREADS = 384;
+// setmaxnreg split of the launch budget (NUM_THREADS x LAUNCH_REGS):
+// 2 softmax warpgroups x 128 x SOFTMAX_REGS + 128 x CONTROL_REGS.
+constexpr int LAUNCH_REGS = 168;
+constexpr int SOFTMAX_REGS = 224;
+constexpr int CONTROL_REGS = 56;
+static_assert(256 * SOFTMAX_REGS + 128 * CONTROL_REGS <= NUM_THREADS * LAUNCH_REGS,
+              "register split exceeds the launch budget");
+// Bounded waits, in SM cycles: about 2 s (0.2 s for the drain after a
+// timeout) at the 1.965 GHz maximum clock, longer at lower clocks.
+constexpr uint64_t WAIT_LIMIT_CYCLES = 4000000000ull;
+constexpr uint64_t DRAIN_LIMIT_CYCLES = 400000000ull;
+#ifndef WMKV_RESCALE_THRESHOLD
+#define WMKV_RESCALE_THRESHOLD 8.0f
+#endif
+// log2 units: O and l are rescaled only when the row max grows by more than 2^8
+constexpr float RESCALE_THRESHOLD = WMKV_RESCALE_THRESHOLD;
 
 template <int D>
 struct Cfg {
   static constexpr int SUB = D / 64;             // 64-column (128-byte) sub-tiles per row
   static constexpr int SUB_BYTES = BN * 128;     // one sub-tile: 128 rows x 128 B
   static constexpr int TILE_BYTES = SUB * SUB_BYTES;
-  static constexpr int NS = (D == 64) ? 4 : 2;   // K/V ring stages
+  // K and V rings.  A K stage is released as soon as its S MMA completes, a
+  // V stage after its P.V; the producer keeps K two tiles ahead of V.
+  static constexpr int NK = (D == 64) ? 5 : 3;
+  static constexpr int NV = (D == 64) ? 4 : 3;
+  static constexpr int K_AHEAD = 2;
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + TILE_BYTES;
-  static constexpr int V_OFF = K_OFF + NS * TILE_BYTES;
-  static constexpr int BAR_OFF = V_OFF + NS * TILE_BYTES;
+  static constexpr int V_OFF = K_OFF + NK * TILE_BYTES;
+  static constexpr int BAR_OFF = V_OFF + NV * TILE_BYTES;
   // barrier indices
   static constexpr int B_Q = 0;
   static constexpr int B_KFULL = 1;
-  static constexpr int B_VFULL = B_KFULL + NS;
-  static constexpr int B_EMPTY = B_VFULL + NS;
-  static constexpr int B_SFULL = B_EMPTY + NS;   // 2
-  static constexpr int B_PFULL = B_SFULL + 2;    // 2
-  static constexpr int B_OFINAL = B_PFULL + 2;
-  static constexpr int B_DRAIN = B_OFINAL + 1;
-  static constexpr int NBAR = B_DRAIN + 1;
+  static constexpr int B_KEMPTY = B_KFULL + NK;
+  static constexpr int B_VFULL = B_KEMPTY + NK;
+  static constexpr int B_VEMPTY = B_VFULL + NV;
+  static constexpr int B_SFULL = B_VEMPTY + NV;  // 2
+  static constexpr int B_SFREE = B_SFULL + 2;    // 2
+  static constexpr int B_PFULL = B_SFREE + 2;    // 2
+  static constexpr int B_ODONE = B_PFULL + 2;    // 2
+  static constexpr int B_OFINAL = B_ODONE + 2;
+  static constexpr int B_DRAIN = B_OFINAL + 1;   // 2: one per MMA issuer
+  static constexpr int NBAR = B_DRAIN + 2;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;   // [0] tmem base, [1] abort
-  static constexpr int XCH_OFF = MISC_OFF + 16;         // m[2][BM], l[2][BM]
-  static constexpr int SMEM_BYTES = XCH_OFF + 4 * BM * 4;
+  // m[2][BM], l[2][BM] for the final merge; they reuse the Q tile, which no
+  // MMA reads any more once the last P.V has completed
+  static constexpr int XCH_OFF = Q_OFF;
+  static constexpr int SMEM_BYTES = MISC_OFF + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;  // 1024-byte alignment slack
-  // TMEM columns: S0, S1 (128 fp32 each), O0, O1 (D fp32 each)
-  static constexpr uint32_t S0_COL = 0, S1_COL = 128, O0_COL = 256, O1_COL = 256 + D;
+  // TMEM columns
+  static constexpr bool P_SEP = (D == 64);
+  // d = 64: S and P.V MMAs come from two issuing threads (their MMAs are short,
+  // so per-tile waits and commits would otherwise leave the tensor core idle);
+  // d = 128: one issuer, which keeps S_{j+2} behind P_j.V_j in issue order.
+  static constexpr bool TWO_ISSUERS = P_SEP;
+  static constexpr uint32_t S_COL0 = 0, S_COL1 = 128;
+  static constexpr uint32_t P_COL0 = P_SEP ? 256 : S_COL0;
+  static constexpr uint32_t P_COL1 = P_SEP ? 320 : S_COL1;
+  static constexpr uint32_t O_COL0 = P_SEP ? 384 : 256;
+  static constexpr uint32_t O_COL1 = O_COL0 + D;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, false, false);
   static constexpr uint32_t IDESC_O = idesc_bf16_f32(BM, D, false, true);
   static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory budget");
-  static_assert(O1_COL + D <= TMEM_COLS, "TMEM budget");
+  static_assert(O_COL1 + D <= TMEM_COLS, "TMEM budget");
 };
+
+// Of every 8 column pairs of a score row, this many get their exponential
+// from the FMA-pipe polynomial instead of MUFU.EX2 (measured on B200: 3 is
+// best for d = 64, where exponentials per FLOP are twice as frequent; 0 for
+// d = 128).
+#ifndef WMKV_POLY_PAIRS_PER_8
+#define WMKV_POLY_PAIRS_PER_8 -1
+#endif
+template <int D>
+constexpr int poly_pairs_per_8() {
+  return WMKV_POLY_PAIRS_PER_8 >= 0 ? WMKV_POLY_PAIRS_PER_8 : (D == 64 ? 3 : 0);
+}
 
 struct AttendParams {
   CUtensorMap tm_q;
@@ -91,6 +152,28 @@ struct AttendParams {
 
 __device__ __forceinline__ void record_timeout(int* status) {
   if (status) atomicExch(status, DEV_TIMEOUT);
+}
+
+// MMA issue helpers.  Descriptors are built once; the start-address field
+// (bits 0-13, in 16-byte units) is advanced by compile-time offsets, so the
+// issuing thread spends its cycles on tcgen05.mma and not on descriptor math.
+template <int D>
+__device__ __forceinline__ void issue_s(uint64_t dq, uint64_t dk, uint32_t d_s) {
+  using C = Cfg<D>;
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint64_t off = uint64_t(((kk / 4) * C::SUB_BYTES + (kk % 4) * 32) >> 4);
+    mma_ss(d_s, dq + off, dk + off, C::IDESC_S, kk > 0 ? 1u : 0u);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void issue_pv(uint64_t dv, uint32_t p_tmem, uint32_t d_o, uint32_t accumulate) {
+  using C = Cfg<D>;
+#pragma unroll
+  for (int kk = 0; kk < BN / 16; ++kk)
+    mma_ts(d_o, p_tmem + kk * 8, dv + uint64_t((kk * 2048) >> 4), C::IDESC_O,
+           (accumulate | uint32_t(kk > 0)));
 }
 
 template <int D>
@@ -114,17 +197,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
 
   if (threadIdx.x == 0) {
     mbar_init(bar(C::B_Q), 1);
-    for (int s = 0; s < C::NS; ++s) {
+    for (int s = 0; s < C::NK; ++s) {
       mbar_init(bar(C::B_KFULL + s), 1);
+      mbar_init(bar(C::B_KEMPTY + s), 1);
+    }
+    for (int s = 0; s < C::NV; ++s) {
       mbar_init(bar(C::B_VFULL + s), 1);
-      mbar_init(bar(C::B_EMPTY + s), 1);
+      mbar_init(bar(C::B_VEMPTY + s), 1);
     }
     for (int g = 0; g < 2; ++g) {
       mbar_init(bar(C::B_SFULL + g), 1);
+      mbar_init(bar(C::B_SFREE + g), 128);
       mbar_init(bar(C::B_PFULL + g), 128);
+      mbar_init(bar(C::B_ODONE + g), 1);
     }
     mbar_init(bar(C::B_OFINAL), 1);
     mbar_init(bar(C::B_DRAIN), 1);
+    mbar_init(bar(C::B_DRAIN + 1), 1);
     misc[1] = 0;
     fence_mbar_init();
   }
@@ -137,7 +226,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
   tc_fence_after();
   const uint32_t tmem = misc[0];
 
-  if (warp == 8) {
+  // Each warpgroup re-sizes its registers at the top of its own branch (the
+  // allocator gives code below a join the smaller of the two limits).
+  if (warp >= 8) {
+   regs_dec<CONTROL_REGS>();
+   if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&p.tm_q);
@@ -147,116 +240,187 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
       for (int s = 0; s < C::SUB; ++s)
         tma_load_3d(sbase + C::Q_OFF + s * C::SUB_BYTES, &p.tm_q, s * 64, head, q_tile * BM,
                     bar(C::B_Q));
-      int issued = 0;
-      for (int j = 0; j < nkv; ++j) {
-        const int st = j % C::NS;
-        const int round = j / C::NS;
-        if (round > 0 && !mbar_wait_bounded(bar(C::B_EMPTY + st), (round - 1) & 1, abort_flag,
-                                            WAIT_LIMIT_NS))
-          break;
-        mbar_expect_tx(bar(C::B_KFULL + st), C::TILE_BYTES);
-        for (int s = 0; s < C::SUB; ++s)
-          tma_load_3d(sbase + C::K_OFF + st * C::TILE_BYTES + s * C::SUB_BYTES, &p.tm_k, s * 64,
-                      head, j * BN, bar(C::B_KFULL + st));
-        mbar_expect_tx(bar(C::B_VFULL + st), C::TILE_BYTES);
-        for (int s = 0; s < C::SUB; ++s)
-          tma_load_3d(sbase + C::V_OFF + st * C::TILE_BYTES + s * C::SUB_BYTES, &p.tm_v, s * 64,
-                      head, j * BN, bar(C::B_VFULL + st));
-        issued = j + 1;
+      // K tile i and V tile i - K_AHEAD per step; each waits for its own ring slot
+      int k_issued = 0, v_issued = 0;
+      for (int i = 0; i < nkv + C::K_AHEAD; ++i) {
+        if (i < nkv) {
+          const int st = i % C::NK;
+          if (i >= C::NK && !mbar_wait_bounded(bar(C::B_KEMPTY + st), ((i / C::NK) - 1) & 1,
+                                               abort_flag, WAIT_LIMIT_CYCLES))
+            break;
+          mbar_expect_tx(bar(C::B_KFULL + st), C::TILE_BYTES);
+          for (int s = 0; s < C::SUB; ++s)
+            tma_load_3d(sbase + C::K_OFF + st * C::TILE_BYTES + s * C::SUB_BYTES, &p.tm_k, s * 64,
+                        head, i * BN, bar(C::B_KFULL + st));
+          k_issued = i + 1;
+        }
+        const int jv = i - C::K_AHEAD;
+        if (jv >= 0 && jv < nkv) {
+          const int st = jv % C::NV;
+          if (jv >= C::NV && !mbar_wait_bounded(bar(C::B_VEMPTY + st), ((jv / C::NV) - 1) & 1,
+                                                abort_flag, WAIT_LIMIT_CYCLES))
+            break;
+          mbar_expect_tx(bar(C::B_VFULL + st), C::TILE_BYTES);
+          for (int s = 0; s < C::SUB; ++s)
+            tma_load_3d(sbase + C::V_OFF + st * C::TILE_BYTES + s * C::SUB_BYTES, &p.tm_v, s * 64,
+                        head, jv * BN, bar(C::B_VFULL + st));
+          v_issued = jv + 1;
+        }
       }
       if (*abort_flag) {
         // Let the copies this thread started land before the CTA exits.
         volatile int no_abort = 0;
-        for (int j = issued - C::NS < 0 ? 0 : issued - C::NS; j < issued; ++j) {
-          const int st = j % C::NS;
-          const uint32_t par = (j / C::NS) & 1;
-          mbar_wait_bounded(bar(C::B_KFULL + st), par, &no_abort, DRAIN_LIMIT_NS);
-          mbar_wait_bounded(bar(C::B_VFULL + st), par, &no_abort, DRAIN_LIMIT_NS);
-        }
+        for (int i = k_issued - C::NK < 0 ? 0 : k_issued - C::NK; i < k_issued; ++i)
+          mbar_wait_bounded(bar(C::B_KFULL + i % C::NK), (i / C::NK) & 1, &no_abort,
+                            DRAIN_LIMIT_CYCLES);
+        for (int i = v_issued - C::NV < 0 ? 0 : v_issued - C::NV; i < v_issued; ++i)
+          mbar_wait_bounded(bar(C::B_VFULL + i % C::NV), (i / C::NV) & 1, &no_abort,
+                            DRAIN_LIMIT_CYCLES);
       }
     }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 9 || warp == 10) {
+    // ------------------------------------------------------------ MMA issuers
+    // Two issuing threads share the tensor core: warp 9 issues S = Q K^T,
+    // warp 10 issues O += P V, so that each thread's barrier waits and
+    // commits overlap with the other's MMAs.  A commit tracks only the
+    // committing thread's own MMAs.
     if (lane == 0) {
-      bool ok = mbar_wait_bounded(bar(C::B_Q), 0, abort_flag, WAIT_LIMIT_NS);
-      tc_fence_after();
-      for (int j = 0; ok && j <= nkv; ++j) {
-        if (j < nkv) {
-          const int st = j % C::NS;
-          const int g = j & 1;
-          if (!mbar_wait_bounded(bar(C::B_KFULL + st), (j / C::NS) & 1, abort_flag, WAIT_LIMIT_NS)) {
-            ok = false;
-            break;
+      constexpr uint64_t TILE16 = C::TILE_BYTES >> 4;
+      bool ok = true;
+      if (!C::TWO_ISSUERS) {
+        // d = 128: one thread issues everything in order; S_{j+2} follows
+        // P_j.V_j in the MMA pipe, which is what lets P overwrite S_j in place
+        if (warp == 9) {
+          const uint64_t dq = sdesc_sw128(sbase + C::Q_OFF, 16, 1024);
+          const uint64_t dk0 = sdesc_sw128(sbase + C::K_OFF, 16, 1024);
+          const uint64_t dv0 = sdesc_sw128(sbase + C::V_OFF, C::SUB_BYTES, 1024);
+          uint32_t k_st = 0, k_ph = 0, v_st = 0, v_ph = 0, pf_ph = 0;
+          ok = mbar_spin_bounded(bar(C::B_Q), 0, abort_flag, WAIT_LIMIT_CYCLES);
+          auto do_s = [&](int g) -> bool {
+            if (!mbar_spin_bounded(bar(C::B_KFULL + k_st), k_ph, abort_flag, WAIT_LIMIT_CYCLES))
+              return false;
+            tc_fence_after();
+            issue_s<D>(dq, dk0 + k_st * TILE16, tmem + (g ? C::S_COL1 : C::S_COL0));
+            tc_commit(bar(C::B_SFULL + g));
+            tc_commit(bar(C::B_KEMPTY + k_st));
+            if (++k_st == C::NK) { k_st = 0; k_ph ^= 1; }
+            return true;
+          };
+          for (int j = 0; ok && j < 2 && j < nkv; ++j) ok = do_s(j);
+          for (int j = 0; ok && j < nkv; ++j) {
+            const int g = j & 1;
+            if (!mbar_spin_bounded(bar(C::B_PFULL + g), (pf_ph >> g) & 1, abort_flag,
+                                   WAIT_LIMIT_CYCLES) ||
+                !mbar_spin_bounded(bar(C::B_VFULL + v_st), v_ph, abort_flag, WAIT_LIMIT_CYCLES)) {
+              ok = false;
+              break;
+            }
+            pf_ph ^= 1u << g;
+            tc_fence_after();
+            issue_pv<D>(dv0 + v_st * TILE16, tmem + (g ? C::P_COL1 : C::P_COL0),
+                        tmem + (g ? C::O_COL1 : C::O_COL0), j >= 2 ? 1u : 0u);
+            tc_commit(bar(C::B_ODONE + g));
+            tc_commit(bar(C::B_VEMPTY + v_st));
+            if (++v_st == C::NV) { v_st = 0; v_ph ^= 1; }
+            if (j + 2 < nkv && !(ok = do_s(g))) break;
           }
-          tc_fence_after();
-          const uint32_t k_tile = sbase + C::K_OFF + st * C::TILE_BYTES;
-          const uint32_t d_s = tmem + (g ? C::S1_COL : C::S0_COL);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk / 4) * C::SUB_BYTES + (kk % 4) * 32;
-            const uint64_t a = sdesc_sw128(sbase + C::Q_OFF + off, 16, 1024);
-            const uint64_t b = sdesc_sw128(k_tile + off, 16, 1024);
-            mma_ss(d_s, a, b, C::IDESC_S, kk > 0 ? 1u : 0u);
-          }
-          tc_commit(bar(C::B_SFULL + g));
+          if (ok) tc_commit(bar(C::B_OFINAL));
         }
-        if (j >= 1) {
-          const int jp = j - 1;
-          const int gp = jp & 1;
-          const int stp = jp % C::NS;
-          if (!mbar_wait_bounded(bar(C::B_PFULL + gp), (jp / 2) & 1, abort_flag, WAIT_LIMIT_NS) ||
-              !mbar_wait_bounded(bar(C::B_VFULL + stp), (jp / C::NS) & 1, abort_flag,
-                                 WAIT_LIMIT_NS)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t v_tile = sbase + C::V_OFF + stp * C::TILE_BYTES;
-          const uint32_t p_tmem = tmem + (gp ? C::S1_COL : C::S0_COL);
-          const uint32_t d_o = tmem + (gp ? C::O1_COL : C::O0_COL);
-#pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk) {
-            const uint64_t b = sdesc_sw128(v_tile + kk * 2048, C::SUB_BYTES, 1024);
-            mma_ts(d_o, p_tmem + kk * 8, b, C::IDESC_O, (jp >= 2 || kk > 0) ? 1u : 0u);
-          }
-          tc_commit(bar(C::B_EMPTY + stp));
-        }
-      }
-      if (ok) {
-        tc_commit(bar(C::B_OFINAL));
       } else {
+      if (warp == 9) {
+        const uint64_t dq = sdesc_sw128(sbase + C::Q_OFF, 16, 1024);
+        const uint64_t dk0 = sdesc_sw128(sbase + C::K_OFF, 16, 1024);
+        uint32_t k_st = 0, k_ph = 0;  // ring slot / phase of the next K tile
+        uint32_t fr_ph = 0;           // bit g: phase of the barrier that frees S_g
+        ok = mbar_spin_bounded(bar(C::B_Q), 0, abort_flag, WAIT_LIMIT_CYCLES);
+        for (int j = 0; ok && j < nkv; ++j) {
+          const int g = j & 1;
+          if (j >= 2) {
+            // S_g is free once the warpgroup has read S_{j-2} (d = 64: P has its
+            // own columns) or once P_{j-2}.V_{j-2} has completed (d = 128: P
+            // overwrote S_{j-2})
+            const int fb = C::P_SEP ? C::B_SFREE + g : C::B_ODONE + g;
+            if (!mbar_spin_bounded(bar(fb), (fr_ph >> g) & 1, abort_flag, WAIT_LIMIT_CYCLES)) {
+              ok = false;
+              break;
+            }
+            fr_ph ^= 1u << g;
+          }
+          if (!mbar_spin_bounded(bar(C::B_KFULL + k_st), k_ph, abort_flag, WAIT_LIMIT_CYCLES)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_s<D>(dq, dk0 + k_st * TILE16, tmem + (g ? C::S_COL1 : C::S_COL0));
+          tc_commit(bar(C::B_SFULL + g));
+          tc_commit(bar(C::B_KEMPTY + k_st));
+          if (++k_st == C::NK) { k_st = 0; k_ph ^= 1; }
+        }
+      } else if (warp == 10) {
+        const uint64_t dv0 = sdesc_sw128(sbase + C::V_OFF, C::SUB_BYTES, 1024);
+        uint32_t v_st = 0, v_ph = 0;  // ring slot / phase of the next V tile
+        uint32_t pf_ph = 0;           // bit g: phase of P_full[g]
+        for (int j = 0; ok && j < nkv; ++j) {
+          const int g = j & 1;
+          if (!mbar_spin_bounded(bar(C::B_PFULL + g), (pf_ph >> g) & 1, abort_flag,
+                                 WAIT_LIMIT_CYCLES) ||
+              !mbar_spin_bounded(bar(C::B_VFULL + v_st), v_ph, abort_flag, WAIT_LIMIT_CYCLES)) {
+            ok = false;
+            break;
+          }
+          pf_ph ^= 1u << g;
+          tc_fence_after();
+          issue_pv<D>(dv0 + v_st * TILE16, tmem + (g ? C::P_COL1 : C::P_COL0),
+                      tmem + (g ? C::O_COL1 : C::O_COL0), j >= 2 ? 1u : 0u);
+          tc_commit(bar(C::B_ODONE + g));
+          tc_commit(bar(C::B_VEMPTY + v_st));
+          if (++v_st == C::NV) { v_st = 0; v_ph ^= 1; }
+        }
+        if (ok) tc_commit(bar(C::B_OFINAL));
+      }
+      }
+      if ((warp == 9 || warp == 10) && !ok) {
+        // let this thread's MMAs finish before TMEM is released
         volatile int no_abort = 0;
-        tc_commit(bar(C::B_DRAIN));
-        mbar_wait_bounded(bar(C::B_DRAIN), 0, &no_abort, DRAIN_LIMIT_NS);
+        const int db = warp == 9 ? C::B_DRAIN : C::B_DRAIN + 1;
+        tc_commit(bar(db));
+        mbar_wait_bounded(bar(db), 0, &no_abort, DRAIN_LIMIT_CYCLES);
       }
     }
+   }
   } else {
+    regs_inc<SOFTMAX_REGS>();
     // ------------------------------------------------------------ softmax
     const int wg = warp / 4;
     const int wq = warp % 4;
     const int row = wq * 32 + lane;
     const uint32_t lane_off = uint32_t(wq * 32) << 16;
-    const uint32_t s_addr = tmem + lane_off + (wg ? C::S1_COL : C::S0_COL);
-    const uint32_t o_addr = tmem + lane_off + (wg ? C::O1_COL : C::O0_COL);
+    const uint32_t s_addr = tmem + lane_off + (wg ? C::S_COL1 : C::S_COL0);
+    const uint32_t p_addr = tmem + lane_off + (wg ? C::P_COL1 : C::P_COL0);
+    const uint32_t o_addr = tmem + lane_off + (wg ? C::O_COL1 : C::O_COL0);
     const float sl2 = p.scale_log2;
-    float m_run = -INFINITY;
+    float m_ref = -INFINITY;  // exponent reference (log2 units)
     float l_run = 0.f;
     bool ok = true;
     int n = 0;
     for (int j = wg; j < nkv; j += 2, ++n) {
-      ok = mbar_wait_bounded(bar(C::B_SFULL + wg), n & 1, abort_flag, WAIT_LIMIT_NS);
+      ok = mbar_wait_bounded(bar(C::B_SFULL + wg), n & 1, abort_flag, WAIT_LIMIT_CYCLES);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      uint32_t sr[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, sr[c]);
+      uint32_t sr[128];
+      tmem_ld32_at<0>(s_addr, sr);
+      tmem_ld32_at<32>(s_addr + 32, sr);
+      tmem_ld32_at<64>(s_addr + 64, sr);
+      tmem_ld32_at<96>(s_addr + 96, sr);
       tmem_wait_ld();
+      if (C::P_SEP) {
+        tc_fence_before();
+        mbar_arrive(bar(C::B_SFREE + wg));
+      }
       float s[128];
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(sr[c][i]);
+      for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
       if (j == nkv - 1) {
         const int valid = static_cast<int>(p.lk - int64_t(j) * BN);
         if (valid < BN) {
@@ -265,47 +429,95 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
             if (c >= valid) s[c] = -INFINITY;
         }
       }
-      float mx = s[0];
+      // row max: four independent chains of three-input max
+      float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
-      const float m_new = fmaxf(m_run, mx * sl2);
-      const float alpha = ex2_approx(m_run - m_new);
-      const float neg_m = -m_new;
-      float sum = 0.f;
-      uint32_t pk[2][32];
-#pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float p0 = ex2_approx(fmaf(s[2 * c], sl2, neg_m));
-        const float p1 = ex2_approx(fmaf(s[2 * c + 1], sl2, neg_m));
-        sum += p0 + p1;
-        pk[c / 32][c % 32] = pack_bf16x2(p0, p1);
+      for (int c = 4; c < 128; c += 8) {
+        mx0 = fmax3(mx0, s[c + 0], s[c + 4]);
+        mx1 = fmax3(mx1, s[c + 1], s[c + 5]);
+        mx2 = fmax3(mx2, s[c + 2], s[c + 6]);
+        mx3 = fmax3(mx3, s[c + 3], s[c + 7]);
       }
-      l_run = l_run * alpha + sum;
-      m_run = m_new;
-      tmem_st32(s_addr, pk[0]);
-      tmem_st32(s_addr + 32, pk[1]);
-      if (n > 0 && __any_sync(0xffffffffu, alpha < 1.f)) {
+      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+      float alpha = 1.f;
+      bool grow = false;
+      if (n == 0) {
+        m_ref = m_tile;
+      } else if (m_tile > m_ref + RESCALE_THRESHOLD) {
+        alpha = ex2_approx(m_ref - m_tile);
+        m_ref = m_tile;
+        grow = true;
+      }
+      // p = 2^(s * sl2 - m_ref), packed to bf16 pairs
+      const f2 scale2 = f2_make(sl2, sl2);
+      const f2 negm2 = f2_make(-m_ref, -m_ref);
+      f2 acc0 = f2_make(0.f, 0.f), acc1 = acc0, acc2 = acc0, acc3 = acc0;
+      uint32_t pk[64];
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t orr[32];
-          tmem_ld32(o_addr + c * 32, orr);
-          tmem_wait_ld();
+      for (int pp = 0; pp < 64; ++pp) {
+        const f2 x = f2_fma(f2_make(s[2 * pp], s[2 * pp + 1]), scale2, negm2);
+        f2 e;
+        if ((pp % 8) >= 8 - poly_pairs_per_8<D>()) {
+          e = exp2_poly2(x);
+        } else {
+          float x0, x1;
+          f2_split(x, x0, x1);
+          e = f2_make(ex2_approx(x0), ex2_approx(x1));
+        }
+        switch (pp % 4) {
+          case 0: acc0 = f2_add(acc0, e); break;
+          case 1: acc1 = f2_add(acc1, e); break;
+          case 2: acc2 = f2_add(acc2, e); break;
+          default: acc3 = f2_add(acc3, e); break;
+        }
+        float e0, e1;
+        f2_split(e, e0, e1);
+        pk[pp] = pack_bf16x2(e0, e1);
+      }
+      const f2 acc = f2_add(f2_add(acc0, acc1), f2_add(acc2, acc3));
+      float a_lo, a_hi;
+      f2_split(acc, a_lo, a_hi);
+      // l is rescaled by alpha (1 unless the reference grew) before this tile's sum
+      l_run = l_run * alpha + (a_lo + a_hi);
+      if (n > 0) {
+        // P.V of this warpgroup's previous tile has finished: O is stable, P is free
+        ok = mbar_wait_bounded(bar(C::B_ODONE + wg), (n - 1) & 1, abort_flag, WAIT_LIMIT_CYCLES);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
-          tmem_st32(o_addr + c * 32, orr);
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t orr[32];
+            tmem_ld32(o_addr + c * 32, orr);
+            tmem_wait_ld();
+            const f2 a2 = f2_make(alpha, alpha);
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+              f2 v = f2_make(__uint_as_float(orr[i]), __uint_as_float(orr[i + 1]));
+              v = f2_mul(v, a2);
+              float lo, hi;
+              f2_split(v, lo, hi);
+              orr[i] = __float_as_uint(lo);
+              orr[i + 1] = __float_as_uint(hi);
+            }
+            tmem_st32(o_addr + c * 32, orr);
+          }
         }
       }
+      tmem_st32_at<0>(p_addr, pk);
+      tmem_st32_at<32>(p_addr + 32, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(C::B_PFULL + wg));
     }
     // all P.V products must have landed before O is read
     if (ok) {
-      ok = mbar_wait_bounded(bar(C::B_OFINAL), 0, abort_flag, WAIT_LIMIT_NS);
+      ok = mbar_wait_bounded(bar(C::B_OFINAL), 0, abort_flag, WAIT_LIMIT_CYCLES);
       ok = __all_sync(0xffffffffu, ok);
     }
     tc_fence_after();
-    xch_m[wg * BM + row] = m_run;
+    xch_m[wg * BM + row] = m_ref;
     xch_l[wg * BM + row] = l_run;
     named_bar_sync(1, 256);
     if (ok && !*abort_flag) {
@@ -319,8 +531,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
       const bool has1 = nkv > 1;
       const int64_t qrow = int64_t(q_tile) * BM + row;
       __nv_bfloat16* orow = p.o + (qrow * p.heads + head) * D;
-      const uint32_t o0 = tmem + lane_off + C::O0_COL;
-      const uint32_t o1 = tmem + lane_off + C::O1_COL;
+      const uint32_t o0 = tmem + lane_off + C::O_COL0;
+      const uint32_t o1 = tmem + lane_off + C::O_COL1;
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
         const int col = wg * (D / 2) + c * 32;
@@ -397,6 +609,11 @@ cudaError_t launch_d(const AttendParams& prm, int64_t lq, int heads, cudaStream_
   std::call_once(once, [] {
     attr_err = cudaFuncSetAttribute(attend_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     C::SMEM_ALLOC);
+    // setmaxnreg.inc waits until registers are free: the launch must carry
+    // exactly the budget the split assumes, or the kernel is not launched.
+    cudaFuncAttributes fa;
+    if (attr_err == cudaSuccess) attr_err = cudaFuncGetAttributes(&fa, attend_kernel<D>);
+    if (attr_err == cudaSuccess && fa.numRegs != LAUNCH_REGS) attr_err = cudaErrorInvalidConfiguration;
   });
   if (attr_err != cudaSuccess) return attr_err;
   dim3 grid(static_cast<unsigned>((lq + BM - 1) / BM), static_cast<unsigned>(heads));

@@ -49,17 +49,47 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Bounded wait: returns false when the phase did not complete within
-// `limit_ns`, or when another thread of the CTA has already given up
-// (`*abort` set).  A kernel that gives up records an error and unwinds
-// instead of spinning forever.
+// `limit_cycles` SM clock cycles, or when another thread of the CTA has
+// already given up (`*abort` set).  A kernel that gives up records an error
+// and unwinds instead of spinning forever.  The cycle counter is cheap to read
+// on the polling path (unlike the global nanosecond timer).
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
-                                                  volatile int* abort, uint64_t limit_ns) {
+                                                  volatile int* abort, uint64_t limit_cycles) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
+  const uint64_t t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (globaltimer_ns() - t0 > limit_ns) {
+    if (static_cast<uint64_t>(clock64()) - t0 > limit_cycles) {
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
+// Non-suspending probe of a phase (used by the single MMA-issuing threads:
+// right after tcgen05.commit a test_wait returns sooner than a try_wait).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded spin on test_wait; same contract as mbar_wait_bounded.
+__device__ __forceinline__ bool mbar_spin_bounded(uint32_t bar, uint32_t parity,
+                                                  volatile int* abort, uint64_t limit_cycles) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = clock64();
+  while (true) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (static_cast<uint64_t>(clock64()) - t0 > limit_cycles) {
       *abort = 1;
       return false;
     }
@@ -185,6 +215,39 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
                WMKV_W32(r)
                : "memory");
 }
+// The same, writing/reading 32 consecutive entries of a larger register array
+// at a compile-time offset (keeps the array in registers: no pointer casts).
+#define WMKV_RO32(a, o) \
+  "=r"(a[o + 0]), "=r"(a[o + 1]), "=r"(a[o + 2]), "=r"(a[o + 3]), "=r"(a[o + 4]), \
+  "=r"(a[o + 5]), "=r"(a[o + 6]), "=r"(a[o + 7]), "=r"(a[o + 8]), "=r"(a[o + 9]), \
+  "=r"(a[o + 10]), "=r"(a[o + 11]), "=r"(a[o + 12]), "=r"(a[o + 13]), "=r"(a[o + 14]), \
+  "=r"(a[o + 15]), "=r"(a[o + 16]), "=r"(a[o + 17]), "=r"(a[o + 18]), "=r"(a[o + 19]), \
+  "=r"(a[o + 20]), "=r"(a[o + 21]), "=r"(a[o + 22]), "=r"(a[o + 23]), "=r"(a[o + 24]), \
+  "=r"(a[o + 25]), "=r"(a[o + 26]), "=r"(a[o + 27]), "=r"(a[o + 28]), "=r"(a[o + 29]), \
+  "=r"(a[o + 30]), "=r"(a[o + 31])
+#define WMKV_WO32(a, o) \
+  "r"(a[o + 0]), "r"(a[o + 1]), "r"(a[o + 2]), "r"(a[o + 3]), "r"(a[o + 4]), "r"(a[o + 5]), \
+  "r"(a[o + 6]), "r"(a[o + 7]), "r"(a[o + 8]), "r"(a[o + 9]), "r"(a[o + 10]), "r"(a[o + 11]), \
+  "r"(a[o + 12]), "r"(a[o + 13]), "r"(a[o + 14]), "r"(a[o + 15]), "r"(a[o + 16]), \
+  "r"(a[o + 17]), "r"(a[o + 18]), "r"(a[o + 19]), "r"(a[o + 20]), "r"(a[o + 21]), \
+  "r"(a[o + 22]), "r"(a[o + 23]), "r"(a[o + 24]), "r"(a[o + 25]), "r"(a[o + 26]), \
+  "r"(a[o + 27]), "r"(a[o + 28]), "r"(a[o + 29]), "r"(a[o + 30]), "r"(a[o + 31])
+
+template <int OFF, int N>
+__device__ __forceinline__ void tmem_ld32_at(uint32_t taddr, uint32_t (&r)[N]) {
+  static_assert(OFF + 32 <= N, "range");
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 " WMKV_P32 ", [%32];"
+               : WMKV_RO32(r, OFF)
+               : "r"(taddr));
+}
+template <int OFF, int N>
+__device__ __forceinline__ void tmem_st32_at(uint32_t taddr, const uint32_t (&r)[N]) {
+  static_assert(OFF + 32 <= N, "range");
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], " WMKV_P32_FROM1 ";" ::"r"(taddr),
+               WMKV_WO32(r, OFF)
+               : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -198,11 +261,83 @@ __device__ __forceinline__ float ex2_approx(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): one instruction, two lanes.
+struct f2 {
+  uint64_t v;
+};
+__device__ __forceinline__ f2 f2_make(float lo, float hi) {
+  f2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r.v) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_split(f2 a, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(a.v));
+}
+__device__ __forceinline__ f2 f2_fma(f2 a, f2 b, f2 c) {
+  f2 r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r.v) : "l"(a.v), "l"(b.v), "l"(c.v));
+  return r;
+}
+__device__ __forceinline__ f2 f2_add(f2 a, f2 b) {
+  f2 r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(a.v), "l"(b.v));
+  return r;
+}
+__device__ __forceinline__ f2 f2_mul(f2 a, f2 b) {
+  f2 r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(a.v), "l"(b.v));
+  return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x on the FMA pipe, for x <= 0 (softmax exponents).  Cody-Waite style
+// reduction x = j + f with j = round(x), f in [-1/2, 1/2] (W. J. Cody and
+// W. Waite, "Software Manual for the Elementary Functions", 1980): j is read
+// from the low mantissa bits of x + 1.5*2^23, 2^f is a cubic minimax
+// polynomial (relative error 7.5e-5 = 2^-13.7 on [-1/2, 1/2]; coefficients
+// fitted for this library by Remez exchange on the relative error), and 2^j
+// is added into the exponent field.  x is clamped at -125 so the result stays
+// a normal float; anything below 2^-125 is negligible next to the row
+// maximum of a softmax (which is 1).  Two lanes per call (f32x2).
+__device__ __forceinline__ f2 exp2_poly2(f2 x) {
+  float x0, x1;
+  f2_split(x, x0, x1);
+  x = f2_make(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const f2 magic = f2_make(12582912.f, 12582912.f);      // 1.5 * 2^23
+  const f2 nmagic = f2_make(-12582912.f, -12582912.f);
+  const f2 t = f2_add(x, magic);                         // round(x) in the low mantissa bits
+  const f2 jf = f2_add(t, nmagic);                       // round(x) as a float
+  const f2 f = f2_fma(jf, f2_make(-1.f, -1.f), x);       // x - round(x), exact
+  f2 p = f2_fma(f, f2_make(0.0551716685295105f, 0.0551716685295105f),
+                f2_make(0.2426111251115799f, 0.2426111251115799f));
+  p = f2_fma(p, f, f2_make(0.6932609677314758f, 0.6932609677314758f));
+  p = f2_fma(p, f, f2_make(0.9999280571937561f, 0.9999280571937561f));
+  float p0, p1, t0, t1;
+  f2_split(p, p0, p1);
+  f2_split(t, t0, t1);
+  return f2_make(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
+                 __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
+}
+
 // Pack two floats to bf16x2 (round to nearest even); `lo` lands in the low half.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// Warpgroup register re-allocation (all 4 warps of a warpgroup execute it).
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {

@@ -18,7 +18,7 @@
 #include <new>
 #include <vector>
 
-#include "../../include/wmkv.h"
+#include "wmkv.h"
 #include "wmkv_internal.h"
 
 struct wm_kvbuf {
