@@ -11,13 +11,12 @@
 //               zero-filled past lk.
 //   warp 9      owns TMEM (512 columns) and issues S_j = Q K_j^T
 //               (tcgen05.mma SS: both operands K-major in smem)
-//   warp 10     issues O_g += P_j V_j (tcgen05.mma TS: P from TMEM, V MN-major
-//               in smem); two issuing threads keep the tensor core fed while
-//               each waits on barriers and commits.  For d = 128 warp 9
-//               issues both, in order.
+//   warps 10/11 issue O_g += P_j V_j for even / odd tiles (tcgen05.mma TS: P
+//               from TMEM, V MN-major in smem); three issuing threads keep the
+//               tensor core fed while each waits on barriers and commits.
+//               For d = 128 warp 9 issues everything, in order.
 //   warps 0-3   softmax warpgroup 0: even key tiles, S0/P0/O0 in TMEM
 //   warps 4-7   softmax warpgroup 1: odd key tiles, S1/P1/O1 in TMEM
-//   warp 11     idle (it completes the control warpgroup 8-11)
 // The control warpgroup gives registers back (setmaxnreg) so that each
 // softmax thread can hold its 128 scores without spilling.  Each softmax
 // thread owns one query row (= one TMEM lane).
@@ -99,9 +98,10 @@ struct Cfg {
   static constexpr int B_SFREE = B_SFULL + 2;    // 2
   static constexpr int B_PFULL = B_SFREE + 2;    // 2
   static constexpr int B_ODONE = B_PFULL + 2;    // 2
-  static constexpr int B_OFINAL = B_ODONE + 2;
-  static constexpr int B_DRAIN = B_OFINAL + 1;   // 2: one per MMA issuer
-  static constexpr int NBAR = B_DRAIN + 2;
+  static constexpr int B_TURN = B_ODONE + 2;    // 2: whose turn it is to run its exponentials
+  static constexpr int B_OFINAL = B_TURN + 2;
+  static constexpr int B_DRAIN = B_OFINAL + 1;   // 3: one per MMA issuer
+  static constexpr int NBAR = B_DRAIN + 3;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;   // [0] tmem base, [1] abort
   // m[2][BM], l[2][BM] for the final merge; they reuse the Q tile, which no
   // MMA reads any more once the last P.V has completed
@@ -124,6 +124,7 @@ struct Cfg {
   static constexpr uint32_t IDESC_O = idesc_bf16_f32(BM, D, false, true);
   static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory budget");
   static_assert(O_COL1 + D <= TMEM_COLS, "TMEM budget");
+  static_assert(NV % 2 == 0 || !P_SEP, "per-warpgroup P.V issuers need an even V ring");
 };
 
 // Of every 8 column pairs of a score row, this many get their exponential
@@ -133,6 +134,13 @@ struct Cfg {
 #ifndef WMKV_POLY_PAIRS_PER_8
 #define WMKV_POLY_PAIRS_PER_8 -1
 #endif
+// Whether the two softmax warpgroups take turns for their exponential phase
+// (measured: letting them overlap is slightly faster on B200).
+#ifndef WMKV_TAKE_TURNS
+#define WMKV_TAKE_TURNS 0
+#endif
+constexpr bool TAKE_TURNS = WMKV_TAKE_TURNS != 0;
+
 template <int D>
 constexpr int poly_pairs_per_8() {
   return WMKV_POLY_PAIRS_PER_8 >= 0 ? WMKV_POLY_PAIRS_PER_8 : (D == 64 ? 3 : 0);
@@ -210,10 +218,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
       mbar_init(bar(C::B_SFREE + g), 128);
       mbar_init(bar(C::B_PFULL + g), 128);
       mbar_init(bar(C::B_ODONE + g), 1);
+      mbar_init(bar(C::B_TURN + g), 128);
     }
-    mbar_init(bar(C::B_OFINAL), 1);
-    mbar_init(bar(C::B_DRAIN), 1);
-    mbar_init(bar(C::B_DRAIN + 1), 1);
+    // the last P.V of each warpgroup commits once (one issuer per warpgroup
+    // for d = 64; for d = 128 the single issuer commits twice)
+    mbar_init(bar(C::B_OFINAL), 2);
+    for (int i = 0; i < 3; ++i) mbar_init(bar(C::B_DRAIN + i), 1);
     misc[1] = 0;
     fence_mbar_init();
   }
@@ -278,8 +288,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
                             DRAIN_LIMIT_CYCLES);
       }
     }
-  } else if (warp == 9 || warp == 10) {
+  } else if (warp >= 9) {
     // ------------------------------------------------------------ MMA issuers
+    // Waits on the softmax warpgroups (S_free, P_full) suspend the thread
+    // (try_wait) so that the issuers do not take issue slots from the
+    // softmax warps on the same SM sub-partitions; waits on TMA data that
+    // normally has landed already (K_full, V_full) poll (test_wait).
     // Two issuing threads share the tensor core: warp 9 issues S = Q K^T,
     // warp 10 issues O += P V, so that each thread's barrier waits and
     // commits overlap with the other's MMAs.  A commit tracks only the
@@ -309,7 +323,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
           for (int j = 0; ok && j < 2 && j < nkv; ++j) ok = do_s(j);
           for (int j = 0; ok && j < nkv; ++j) {
             const int g = j & 1;
-            if (!mbar_spin_bounded(bar(C::B_PFULL + g), (pf_ph >> g) & 1, abort_flag,
+            if (!mbar_wait_bounded(bar(C::B_PFULL + g), (pf_ph >> g) & 1, abort_flag,
                                    WAIT_LIMIT_CYCLES) ||
                 !mbar_spin_bounded(bar(C::B_VFULL + v_st), v_ph, abort_flag, WAIT_LIMIT_CYCLES)) {
               ok = false;
@@ -324,7 +338,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
             if (++v_st == C::NV) { v_st = 0; v_ph ^= 1; }
             if (j + 2 < nkv && !(ok = do_s(g))) break;
           }
-          if (ok) tc_commit(bar(C::B_OFINAL));
+          if (ok) {
+            tc_commit(bar(C::B_OFINAL));
+            tc_commit(bar(C::B_OFINAL));
+          }
         }
       } else {
       if (warp == 9) {
@@ -340,7 +357,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
             // own columns) or once P_{j-2}.V_{j-2} has completed (d = 128: P
             // overwrote S_{j-2})
             const int fb = C::P_SEP ? C::B_SFREE + g : C::B_ODONE + g;
-            if (!mbar_spin_bounded(bar(fb), (fr_ph >> g) & 1, abort_flag, WAIT_LIMIT_CYCLES)) {
+            if (!mbar_wait_bounded(bar(fb), (fr_ph >> g) & 1, abort_flag, WAIT_LIMIT_CYCLES)) {
               ok = false;
               break;
             }
@@ -356,33 +373,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
           tc_commit(bar(C::B_KEMPTY + k_st));
           if (++k_st == C::NK) { k_st = 0; k_ph ^= 1; }
         }
-      } else if (warp == 10) {
+      } else {
+        // warp 10: P.V of even tiles, warp 11: odd tiles (each issuing thread
+        // keeps its own V slots: the V ring has an even number of stages)
+        const int g = warp - 10;
         const uint64_t dv0 = sdesc_sw128(sbase + C::V_OFF, C::SUB_BYTES, 1024);
-        uint32_t v_st = 0, v_ph = 0;  // ring slot / phase of the next V tile
-        uint32_t pf_ph = 0;           // bit g: phase of P_full[g]
-        for (int j = 0; ok && j < nkv; ++j) {
-          const int g = j & 1;
-          if (!mbar_spin_bounded(bar(C::B_PFULL + g), (pf_ph >> g) & 1, abort_flag,
-                                 WAIT_LIMIT_CYCLES) ||
+        const uint32_t p_tm = tmem + (g ? C::P_COL1 : C::P_COL0);
+        const uint32_t o_tm = tmem + (g ? C::O_COL1 : C::O_COL0);
+        uint32_t pf_ph = 0;
+        for (int j = g; ok && j < nkv; j += 2) {
+          const int v_st = j % C::NV;
+          const uint32_t v_ph = (j / C::NV) & 1;
+          if (!mbar_wait_bounded(bar(C::B_PFULL + g), pf_ph, abort_flag, WAIT_LIMIT_CYCLES) ||
               !mbar_spin_bounded(bar(C::B_VFULL + v_st), v_ph, abort_flag, WAIT_LIMIT_CYCLES)) {
             ok = false;
             break;
           }
-          pf_ph ^= 1u << g;
+          pf_ph ^= 1;
           tc_fence_after();
-          issue_pv<D>(dv0 + v_st * TILE16, tmem + (g ? C::P_COL1 : C::P_COL0),
-                      tmem + (g ? C::O_COL1 : C::O_COL0), j >= 2 ? 1u : 0u);
+          issue_pv<D>(dv0 + v_st * TILE16, p_tm, o_tm, j >= 2 ? 1u : 0u);
           tc_commit(bar(C::B_ODONE + g));
           tc_commit(bar(C::B_VEMPTY + v_st));
-          if (++v_st == C::NV) { v_st = 0; v_ph ^= 1; }
         }
         if (ok) tc_commit(bar(C::B_OFINAL));
       }
       }
-      if ((warp == 9 || warp == 10) && !ok) {
+      if (!ok) {
         // let this thread's MMAs finish before TMEM is released
         volatile int no_abort = 0;
-        const int db = warp == 9 ? C::B_DRAIN : C::B_DRAIN + 1;
+        const int db = C::B_DRAIN + (warp - 9);
         tc_commit(bar(db));
         mbar_wait_bounded(bar(db), 0, &no_abort, DRAIN_LIMIT_CYCLES);
       }
@@ -403,6 +422,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
     float l_run = 0.f;
     bool ok = true;
     int n = 0;
+    uint32_t turn_ph = 0;
+    if (TAKE_TURNS && wg == 1) mbar_arrive(bar(C::B_TURN + 0));  // warpgroup 0 goes first
     for (int j = wg; j < nkv; j += 2, ++n) {
       ok = mbar_wait_bounded(bar(C::B_SFULL + wg), n & 1, abort_flag, WAIT_LIMIT_CYCLES);
       ok = __all_sync(0xffffffffu, ok);
@@ -429,16 +450,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
             if (c >= valid) s[c] = -INFINITY;
         }
       }
-      // row max: four independent chains of three-input max
-      float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+      // row max: eight independent chains of three-input max, then a tree
+      float mx[8];
 #pragma unroll
-      for (int c = 4; c < 128; c += 8) {
-        mx0 = fmax3(mx0, s[c + 0], s[c + 4]);
-        mx1 = fmax3(mx1, s[c + 1], s[c + 5]);
-        mx2 = fmax3(mx2, s[c + 2], s[c + 6]);
-        mx3 = fmax3(mx3, s[c + 3], s[c + 7]);
-      }
-      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+      for (int c = 0; c < 8; ++c) mx[c] = fmax3(s[c], s[c + 8], s[c + 16]);
+#pragma unroll
+      for (int c = 24; c < 120; c += 16)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx[i] = fmax3(mx[i], s[c + i], s[c + 8 + i]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[120 + i]);
+      const float m_tile =
+          fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], fmax3(mx[5], mx[6], mx[7]))) * sl2;
       float alpha = 1.f;
       bool grow = false;
       if (n == 0) {
@@ -447,6 +470,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
         alpha = ex2_approx(m_ref - m_tile);
         m_ref = m_tile;
         grow = true;
+      }
+      if (TAKE_TURNS) {
+        // the two warpgroups take turns for their exponentials
+        ok = mbar_wait_bounded(bar(C::B_TURN + wg), turn_ph, abort_flag, WAIT_LIMIT_CYCLES);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        turn_ph ^= 1;
       }
       // p = 2^(s * sl2 - m_ref), packed to bf16 pairs
       const f2 scale2 = f2_make(sl2, sl2);
@@ -477,6 +507,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
       const f2 acc = f2_add(f2_add(acc0, acc1), f2_add(acc2, acc3));
       float a_lo, a_hi;
       f2_split(acc, a_lo, a_hi);
+      if (TAKE_TURNS && j + 1 < nkv) mbar_arrive(bar(C::B_TURN + (wg ^ 1)));
       // l is rescaled by alpha (1 unless the reference grew) before this tile's sum
       l_run = l_run * alpha + (a_lo + a_hi);
       if (n > 0) {

@@ -297,12 +297,16 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // 2^x on the FMA pipe, for x <= 0 (softmax exponents).  Cody-Waite style
 // reduction x = j + f with j = round(x), f in [-1/2, 1/2] (W. J. Cody and
 // W. Waite, "Software Manual for the Elementary Functions", 1980): j is read
-// from the low mantissa bits of x + 1.5*2^23, 2^f is a cubic minimax
-// polynomial (relative error 7.5e-5 = 2^-13.7 on [-1/2, 1/2]; coefficients
-// fitted for this library by Remez exchange on the relative error), and 2^j
-// is added into the exponent field.  x is clamped at -125 so the result stays
-// a normal float; anything below 2^-125 is negligible next to the row
-// maximum of a softmax (which is 1).  Two lanes per call (f32x2).
+// from the low mantissa bits of x + 1.5*2^23, 2^f is a minimax polynomial
+// (coefficients fitted for this library by Remez exchange on the relative
+// error over [-1/2, 1/2]: cubic 7.5e-5 = 2^-13.7, quadratic 1.7e-3 = 2^-9.2,
+// the latter about the size of the bf16 rounding P gets anyway), and 2^j is
+// added into the exponent field.  x is clamped at -125 so the result stays a
+// normal float; anything below 2^-125 is negligible next to the row maximum
+// of a softmax (which is 1).  Two lanes per call (f32x2).
+#ifndef WMKV_POLY_DEGREE
+#define WMKV_POLY_DEGREE 2
+#endif
 __device__ __forceinline__ f2 exp2_poly2(f2 x) {
   float x0, x1;
   f2_split(x, x0, x1);
@@ -312,10 +316,16 @@ __device__ __forceinline__ f2 exp2_poly2(f2 x) {
   const f2 t = f2_add(x, magic);                         // round(x) in the low mantissa bits
   const f2 jf = f2_add(t, nmagic);                       // round(x) as a float
   const f2 f = f2_fma(jf, f2_make(-1.f, -1.f), x);       // x - round(x), exact
+#if WMKV_POLY_DEGREE == 2
+  f2 p = f2_fma(f, f2_make(0.23842893540859222f, 0.23842893540859222f),
+                f2_make(0.7034479975700378f, 0.7034479975700378f));
+  p = f2_fma(p, f, f2_make(1.0004431009292603f, 1.0004431009292603f));
+#else
   f2 p = f2_fma(f, f2_make(0.0551716685295105f, 0.0551716685295105f),
                 f2_make(0.2426111251115799f, 0.2426111251115799f));
   p = f2_fma(p, f, f2_make(0.6932609677314758f, 0.6932609677314758f));
   p = f2_fma(p, f, f2_make(0.9999280571937561f, 0.9999280571937561f));
+#endif
   float p0, p1, t0, t1;
   f2_split(p, p0, p1);
   f2_split(t, t0, t1);

@@ -1,0 +1,199 @@
+"""GPU parity on the large workloads, through the C ABI, against the fp64 oracle.
+
+* full rollout: 28 blocks at the served shape, frames 0..40 from an empty
+  buffer, 4 passes (write + attend) per frame, inputs seeded per
+  (block, frame, pass);
+* batch of 8 independent sessions (28 blocks each) in steady state, K rows
+  scaled by U(0.5, 2) per token;
+* scaled memory: 45x80 grid + 256 summary tokens, Y=2, W=48, 24 heads x 128,
+  28 blocks at t=60, plus the dense full-history baseline (180,000 keys).
+
+Buffers are compared byte for byte; attention on a deterministic row sample
+(rows 0, HW-1, HW, R-1 and 60 seeded rows, all heads) within max-abs 2e-2 and
+relative L2 5e-3.  To keep host generation bounded, the frames that only fill
+a memory up to steady state (batch and scaled workloads) share one record
+across the blocks of a session; every measured frame has per-block data.
+"""
+import numpy as np
+import pytest
+
+import seeded_inputs as si
+from oracle import FrameMemory, Layout, SCALED, SERVED, attend, attend_memory
+from gpu_util import DevicePool, assert_attn_close, host_bits, require_gpu, sample_rows, torch
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+SAMPLED_BLOCKS = (0, 13, 27)
+
+
+@pytest.fixture(scope="module")
+def wm():
+    require_gpu()
+    import kv_memory_attention_b200 as wm
+    return wm
+
+
+@pytest.fixture(scope="module")
+def pool():
+    require_gpu()
+    return DevicePool()
+
+
+def check_block(kv, mem, b, mb):
+    kd, vd = kv.kv_views(b)
+    assert np.array_equal(host_bits(kd), mem.K[mb]), f"K of block {b} differs at t={mem.t}"
+    assert np.array_equal(host_bits(vd), mem.V[mb]), f"V of block {b} differs at t={mem.t}"
+
+
+def test_full_rollout_28_blocks_four_passes(wm, pool):
+    L, B = SERVED, 28
+    kv = wm.KVMemory(B, L.heads, L.d, L.grid_h, L.grid_w, L.X, L.Y, L.W)
+    mem = FrameMemory(L, B, track_records=False)
+    shape = (L.R, L.heads, L.d)
+    full_check_frames = {0, 3, 4, 24, 25, 31, 40}
+    for t in range(41):
+        kv.advance(t)
+        mem.advance(t)
+        assert kv.end() == L.end(t)
+        r0, r1 = L.record_rows(t)
+        for step in range(4):
+            for b in range(B):
+                sk = si.seed_for(3, 0, b, t, step, si.T_K)
+                sv = si.seed_for(3, 0, b, t, step, si.T_V)
+                kd, vd = pool.normal(sk, shape), pool.normal(sv, shape)
+                kv.write_record(b, t, kd, vd)
+                mem.write_record(b, t, si.pool_normal_bf16(sk, shape), si.pool_normal_bf16(sv, shape))
+                kb, vb = kv.kv_views(b)
+                assert torch.equal(kb[r0:r1], kd) and torch.equal(vb[r0:r1], vd), (t, step, b)
+                sq = si.seed_for(3, 0, b, t, step, si.T_Q)
+                o = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+                kv.attend(b, pool.normal(sq, shape), o)
+                if b in SAMPLED_BLOCKS:
+                    rows = sample_rows(L, hash((t, step, b)) & 0xFFFF)
+                    ref = attend_memory(mem, b, si.pool_normal_bf16(sq, shape), rows=rows)
+                    assert_attn_close(host_bits(o)[rows], ref, f"t={t} pass={step} block={b}")
+        torch.cuda.synchronize()
+        for b in (range(B) if t in full_check_frames else SAMPLED_BLOCKS):
+            check_block(kv, mem, b, b)
+    kv.sync_status()
+    kv.close()
+
+
+def test_batch_of_8_sessions_steady_state(wm, pool):
+    L, B, S = SERVED, 28, 8
+    shape = (L.R, L.heads, L.d)
+    sessions = [wm.KVMemory(B, L.heads, L.d, L.grid_h, L.grid_w, L.X, L.Y, L.W) for _ in range(S)]
+    mems = [FrameMemory(L, len(SAMPLED_BLOCKS), track_records=False) for _ in range(S)]
+    # fill to steady state: one record per (session, frame), shared by the blocks
+    for t in range(31):
+        for s, (kv, mem) in enumerate(zip(sessions, mems)):
+            kv.advance(t)
+            mem.advance(t)
+            sk = si.seed_for(4, s, 0, t, 0, si.T_K)
+            ss = si.seed_for(4, s, 0, t, 0, si.T_KSCALE)
+            sv = si.seed_for(4, s, 0, t, 0, si.T_V)
+            k = si.pool_scaled_rows_bf16(sk, ss, L.R, L.heads, L.d)
+            v = si.pool_normal_bf16(sv, shape)
+            kd = torch.from_numpy(k.view(np.int16)).cuda().view(torch.bfloat16)
+            vd = pool.normal(sv, shape)
+            for b in range(B):
+                kv.write_record(b, t, kd, vd)
+            for i in range(len(SAMPLED_BLOCKS)):
+                mem.write_record(i, t, k, v)
+    # measured frames: per-block data, sessions interleaved block by block on one stream
+    for t in (31, 32):
+        for kv, mem in zip(sessions, mems):
+            kv.advance(t)
+            mem.advance(t)
+        for b in range(B):
+            for s, (kv, mem) in enumerate(zip(sessions, mems)):
+                sk = si.seed_for(4, s, b, t, 0, si.T_K)
+                ss = si.seed_for(4, s, b, t, 0, si.T_KSCALE)
+                sv = si.seed_for(4, s, b, t, 0, si.T_V)
+                sq = si.seed_for(4, s, b, t, 0, si.T_Q)
+                k = si.pool_scaled_rows_bf16(sk, ss, L.R, L.heads, L.d)
+                kd = torch.from_numpy(k.view(np.int16)).cuda().view(torch.bfloat16)
+                vd = pool.normal(sv, shape)
+                kv.write_record(b, t, kd, vd)
+                o = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+                kv.attend(b, pool.normal(sq, shape), o)
+                if b in SAMPLED_BLOCKS:
+                    i = SAMPLED_BLOCKS.index(b)
+                    mem.write_record(i, t, k, si.pool_normal_bf16(sv, shape))
+                    rows = sample_rows(L, s * 1000 + b * 10 + t)
+                    ref = attend_memory(mem, i, si.pool_normal_bf16(sq, shape), rows=rows)
+                    assert_attn_close(host_bits(o)[rows], ref, f"session {s} block {b} t={t}")
+                else:
+                    r0, r1 = L.record_rows(t)
+                    kb, vb = kv.kv_views(b)
+                    assert torch.equal(kb[r0:r1], kd) and torch.equal(vb[r0:r1], vd)
+    torch.cuda.synchronize()
+    for kv, mem in zip(sessions, mems):
+        for i, b in enumerate(SAMPLED_BLOCKS):
+            check_block(kv, mem, b, i)
+        kv.sync_status()
+        kv.close()
+
+
+def test_scaled_memory_and_dense_baseline(wm, pool):
+    L, B = SCALED, 28
+    shape = (L.R, L.heads, L.d)
+    kv = wm.KVMemory(B, L.heads, L.d, L.grid_h, L.grid_w, L.X, L.Y, L.W)
+    mem = FrameMemory(L, len(SAMPLED_BLOCKS), track_records=False)
+    for t in range(60):
+        kv.advance(t)
+        mem.advance(t)
+        sk, sv = si.seed_for(5, 0, 0, t, 0, si.T_K), si.seed_for(5, 0, 0, t, 0, si.T_V)
+        kd, vd = pool.normal(sk, shape), pool.normal(sv, shape)
+        for b in range(B):
+            kv.write_record(b, t, kd, vd)
+        k, v = si.pool_normal_bf16(sk, shape), si.pool_normal_bf16(sv, shape)
+        for i in range(len(SAMPLED_BLOCKS)):
+            mem.write_record(i, t, k, v)
+    t = 60
+    kv.advance(t)
+    mem.advance(t)
+    assert kv.end() == 27200
+    for b in range(B):
+        sk, sv, sq = (si.seed_for(5, 0, b, t, 0, x) for x in (si.T_K, si.T_V, si.T_Q))
+        kv.write_record(b, t, pool.normal(sk, shape), pool.normal(sv, shape))
+        o = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+        kv.attend(b, pool.normal(sq, shape), o)
+        if b in SAMPLED_BLOCKS:
+            i = SAMPLED_BLOCKS.index(b)
+            mem.write_record(i, t, si.pool_normal_bf16(sk, shape), si.pool_normal_bf16(sv, shape))
+            rows = sample_rows(L, 500 + b)
+            ref = attend_memory(mem, i, si.pool_normal_bf16(sq, shape), rows=rows)
+            assert_attn_close(host_bits(o)[rows], ref, f"scaled block {b}")
+    torch.cuda.synchronize()
+    for i, b in enumerate(SAMPLED_BLOCKS):
+        check_block(kv, mem, b, i)
+    kv.sync_status()
+    kv.close()
+    del kv
+
+    # dense full-history baseline: HW queries over (W+2) frames of HW raw tokens each
+    frames = L.W + 2
+    lq, lk = L.HW, frames * L.HW
+    raw = (L.HW, L.heads, L.d)
+    seeds_k = [si.seed_for(5, 1, 0, f, 0, si.T_K) for f in range(frames)]
+    seeds_v = [si.seed_for(5, 1, 0, f, 0, si.T_V) for f in range(frames)]
+    sq = si.seed_for(5, 1, 0, frames, 0, si.T_Q)
+    kd = torch.cat([pool.normal(s, raw) for s in seeds_k])
+    vd = torch.cat([pool.normal(s, raw) for s in seeds_v])
+    qd = pool.normal(sq, raw)
+    od = torch.empty(raw, dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    wm.wm_attend_dense(qd, kd, vd, od, lq, lk, L.heads, L.d, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    rows = np.array([0, 1, 127, 128, lq // 2, lq - 1] + list(np.random.default_rng(9).choice(lq, 10, replace=False)))
+    q = si.bf16_bits_to_f64(si.pool_normal_bf16(sq, raw))[rows]
+    k_bits = np.concatenate([si.pool_normal_bf16(s, raw) for s in seeds_k])   # 1.1 GB of bf16
+    v_bits = np.concatenate([si.pool_normal_bf16(s, raw) for s in seeds_v])
+    ref = np.empty((len(rows), L.heads, L.d))
+    for h in range(L.heads):          # one head at a time keeps the fp64 copies small
+        kh = si.bf16_bits_to_f64(k_bits[:, h:h + 1])
+        vh = si.bf16_bits_to_f64(v_bits[:, h:h + 1])
+        ref[:, h:h + 1] = attend(q[:, h:h + 1], kh, vh)
+    assert_attn_close(host_bits(od)[rows], ref, "dense baseline 3600 x 180000")
