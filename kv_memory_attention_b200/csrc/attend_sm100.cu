@@ -98,8 +98,7 @@ struct Cfg {
   static constexpr int B_SFREE = B_SFULL + 2;    // 2
   static constexpr int B_PFULL = B_SFREE + 2;    // 2
   static constexpr int B_ODONE = B_PFULL + 2;    // 2
-  static constexpr int B_TURN = B_ODONE + 2;    // 2: whose turn it is to run its exponentials
-  static constexpr int B_OFINAL = B_TURN + 2;
+  static constexpr int B_OFINAL = B_ODONE + 2;
   static constexpr int B_DRAIN = B_OFINAL + 1;   // 3: one per MMA issuer
   static constexpr int NBAR = B_DRAIN + 3;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;   // [0] tmem base, [1] abort
@@ -134,13 +133,6 @@ struct Cfg {
 #ifndef WMKV_POLY_PAIRS_PER_8
 #define WMKV_POLY_PAIRS_PER_8 -1
 #endif
-// Whether the two softmax warpgroups take turns for their exponential phase
-// (measured: letting them overlap is slightly faster on B200).
-#ifndef WMKV_TAKE_TURNS
-#define WMKV_TAKE_TURNS 0
-#endif
-constexpr bool TAKE_TURNS = WMKV_TAKE_TURNS != 0;
-
 template <int D>
 constexpr int poly_pairs_per_8() {
   return WMKV_POLY_PAIRS_PER_8 >= 0 ? WMKV_POLY_PAIRS_PER_8 : (D == 64 ? 3 : 0);
@@ -203,6 +195,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
   const int head = blockIdx.y;
   const int nkv = static_cast<int>((p.lk + BN - 1) / BN);
 
+  pdl_launch_dependents();
   if (threadIdx.x == 0) {
     mbar_init(bar(C::B_Q), 1);
     for (int s = 0; s < C::NK; ++s) {
@@ -218,7 +211,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
       mbar_init(bar(C::B_SFREE + g), 128);
       mbar_init(bar(C::B_PFULL + g), 128);
       mbar_init(bar(C::B_ODONE + g), 1);
-      mbar_init(bar(C::B_TURN + g), 128);
     }
     // the last P.V of each warpgroup commits once (one issuer per warpgroup
     // for d = 64; for d = 128 the single issuer commits twice)
@@ -231,10 +223,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
     tmem_alloc(smem_u32(misc), C::TMEM_COLS);
     tmem_relinquish();
   }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&p.tm_q);
+    tma_prefetch_desc(&p.tm_k);
+    tma_prefetch_desc(&p.tm_v);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = misc[0];
+  // everything above overlaps the previous kernel in the stream; global
+  // memory (Q, K, V, O, status) is touched only after this point
+  pdl_wait_prior();
 
   // Each warpgroup re-sizes its registers at the top of its own branch (the
   // allocator gives code below a join the smaller of the two limits).
@@ -243,9 +243,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
    if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      tma_prefetch_desc(&p.tm_q);
-      tma_prefetch_desc(&p.tm_k);
-      tma_prefetch_desc(&p.tm_v);
       mbar_expect_tx(bar(C::B_Q), C::TILE_BYTES);
       for (int s = 0; s < C::SUB; ++s)
         tma_load_3d(sbase + C::Q_OFF + s * C::SUB_BYTES, &p.tm_q, s * 64, head, q_tile * BM,
@@ -422,8 +419,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
     float l_run = 0.f;
     bool ok = true;
     int n = 0;
-    uint32_t turn_ph = 0;
-    if (TAKE_TURNS && wg == 1) mbar_arrive(bar(C::B_TURN + 0));  // warpgroup 0 goes first
     for (int j = wg; j < nkv; j += 2, ++n) {
       ok = mbar_wait_bounded(bar(C::B_SFULL + wg), n & 1, abort_flag, WAIT_LIMIT_CYCLES);
       ok = __all_sync(0xffffffffu, ok);
@@ -471,13 +466,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
         m_ref = m_tile;
         grow = true;
       }
-      if (TAKE_TURNS) {
-        // the two warpgroups take turns for their exponentials
-        ok = mbar_wait_bounded(bar(C::B_TURN + wg), turn_ph, abort_flag, WAIT_LIMIT_CYCLES);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        turn_ph ^= 1;
-      }
       // p = 2^(s * sl2 - m_ref), packed to bf16 pairs
       const f2 scale2 = f2_make(sl2, sl2);
       const f2 negm2 = f2_make(-m_ref, -m_ref);
@@ -507,7 +495,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
       const f2 acc = f2_add(f2_add(acc0, acc1), f2_add(acc2, acc3));
       float a_lo, a_hi;
       f2_split(acc, a_lo, a_hi);
-      if (TAKE_TURNS && j + 1 < nkv) mbar_arrive(bar(C::B_TURN + (wg ^ 1)));
       // l is rescaled by alpha (1 unless the reference grew) before this tile's sum
       l_run = l_run * alpha + (a_lo + a_hi);
       if (n > 0) {
@@ -648,8 +635,7 @@ cudaError_t launch_d(const AttendParams& prm, int64_t lq, int heads, cudaStream_
   });
   if (attr_err != cudaSuccess) return attr_err;
   dim3 grid(static_cast<unsigned>((lq + BM - 1) / BM), static_cast<unsigned>(heads));
-  attend_kernel<D><<<grid, NUM_THREADS, C::SMEM_ALLOC, stream>>>(prm);
-  return cudaGetLastError();
+  return launch_pdl(attend_kernel<D>, grid, dim3(NUM_THREADS), C::SMEM_ALLOC, stream, prm);
 }
 
 }  // namespace

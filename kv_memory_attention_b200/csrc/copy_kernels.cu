@@ -11,6 +11,7 @@
 // grid sized to the SM count.
 #include <cuda_runtime.h>
 
+#include "sm100_ptx.cuh"
 #include "wmkv_internal.h"
 
 namespace wmkv {
@@ -51,6 +52,8 @@ __global__ void __launch_bounds__(COPY_THREADS) copy_pair_kernel(const uint4* __
                                                                  uint4* __restrict__ a_dst,
                                                                  uint4* __restrict__ b_dst,
                                                                  int64_t n) {
+  pdl_launch_dependents();
+  pdl_wait_prior();
   const uint4* src = blockIdx.y ? b_src : a_src;
   uint4* dst = blockIdx.y ? b_dst : a_dst;
   const int64_t stride = int64_t(gridDim.x) * COPY_THREADS;
@@ -61,6 +64,8 @@ __global__ void __launch_bounds__(COPY_THREADS) copy_pair_kernel(const uint4* __
 __global__ void __launch_bounds__(COPY_THREADS) evict_kernel(uint8_t* base, int64_t block_stride,
                                                              int64_t tensor_stride, int64_t src_off,
                                                              int64_t dst_off, int64_t n) {
+  pdl_launch_dependents();
+  pdl_wait_prior();
   uint8_t* buf = base + int64_t(blockIdx.y >> 1) * block_stride + int64_t(blockIdx.y & 1) * tensor_stride;
   const uint4* src = reinterpret_cast<const uint4*>(buf + src_off);
   uint4* dst = reinterpret_cast<uint4*>(buf + dst_off);
@@ -96,10 +101,9 @@ cudaError_t launch_copy_pair(const void* a_src, const void* b_src, void* a_dst, 
                              int64_t n16, cudaStream_t stream) {
   if (n16 <= 0) return cudaSuccess;
   dim3 grid(grid_x_for(n16, 2), 2);
-  copy_pair_kernel<<<grid, COPY_THREADS, 0, stream>>>(
-      static_cast<const uint4*>(a_src), static_cast<const uint4*>(b_src), static_cast<uint4*>(a_dst),
-      static_cast<uint4*>(b_dst), n16);
-  return cudaGetLastError();
+  return launch_pdl(copy_pair_kernel, grid, dim3(COPY_THREADS), 0, stream,
+                    static_cast<const uint4*>(a_src), static_cast<const uint4*>(b_src),
+                    static_cast<uint4*>(a_dst), static_cast<uint4*>(b_dst), n16);
 }
 
 cudaError_t launch_evict(void* base, int blocks, int64_t block_stride_bytes,
@@ -107,10 +111,8 @@ cudaError_t launch_evict(void* base, int blocks, int64_t block_stride_bytes,
                          int64_t n16, cudaStream_t stream) {
   if (n16 <= 0 || blocks <= 0) return cudaSuccess;
   dim3 grid(grid_x_for(n16, 2 * blocks), static_cast<unsigned>(2 * blocks));
-  evict_kernel<<<grid, COPY_THREADS, 0, stream>>>(static_cast<uint8_t*>(base), block_stride_bytes,
-                                                  tensor_stride_bytes, src_off_bytes, dst_off_bytes,
-                                                  n16);
-  return cudaGetLastError();
+  return launch_pdl(evict_kernel, grid, dim3(COPY_THREADS), 0, stream, static_cast<uint8_t*>(base),
+                    block_stride_bytes, tensor_stride_bytes, src_off_bytes, dst_off_bytes, n16);
 }
 
 }  // namespace wmkv

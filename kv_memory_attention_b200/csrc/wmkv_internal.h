@@ -3,7 +3,33 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include <utility>
+
 namespace wmkv {
+
+// Launch `kernel` on `stream` with programmatic stream serialization: the
+// kernel may start while its predecessor finishes; every kernel of this
+// library executes griddepcontrol.wait before its first global memory access,
+// so stream order is preserved for all data.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+#ifndef WMKV_NO_PDL
+  cfg.numAttrs = 1;
+#else
+  cfg.numAttrs = 0;
+#endif
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Device-side error word values (written by kernels, read by the host).
 constexpr int DEV_OK = 0;
