@@ -1,9 +1,10 @@
 """Benchmark: steady-state frame-steps of the Summaryformer frame memory on B200.
 
 One step (one "frame") = wm_advance(t) (RAW -> SUM eviction in all 28 blocks)
-followed, for each of the 28 blocks, by wm_write_record (the frame's K/V
-record) and wm_attend (1104 queries x 6,528 keys x 16 heads x 64), at the
-served shape 24x42 + X=96, Y=2, W=24, in steady state (t >= 31).
+followed, for each of the 28 blocks, by wm_write_attend: the frame's K/V
+record written into its slot and the attention of its 1104 queries over the
+6,528 keys (16 heads x 64), in one launch, at the served shape 24x42 + X=96,
+Y=2, W=24, in steady state (t >= 31).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -43,7 +44,7 @@ T_STEADY = 31
 ATTN_FLOP = 4 * R * C * D * HEADS                 # QK^T + PV, multiply-add = 2
 EVICT_BYTES = 2 * 2 * X * HEADS * D * 2 * BLOCKS  # read + write, K and V, all blocks
 WRITE_BYTES = 2 * 2 * R * HEADS * D * 2           # read + write, K and V, one block
-WORKLOAD = (f"served frame-step: advance (evict) + {BLOCKS} x (write_record + attend), "
+WORKLOAD = (f"served frame-step: advance (evict) + {BLOCKS} x write_attend (record write + attend), "
             f"grid {GH}x{GW} + X={X}, Y={Y}, W={W}, {HEADS} heads x {D}, "
             f"{R} queries x {C} keys, steady state t>={T_STEADY}, one session per GPU")
 CONFIG_ID = 3
@@ -183,12 +184,12 @@ def run_ours(args, world, rank, local):
     t = T_STEADY
 
     def step(t, ev=None):
+        # one launch per block: the record write and the attention are fused
         kv.advance(t, stream)
         for b in range(BLOCKS):
-            kv.write_record(b, t, K[b], V[b], stream)
             if ev is not None:
                 ev[b][0].record(stream)
-            kv.attend(b, Q[b], O[b], stream)
+            kv.write_attend(b, t, Q[b], K[b], V[b], O[b], stream)
             if ev is not None:
                 ev[b][1].record(stream)
 
@@ -215,7 +216,7 @@ def run_ours(args, world, rank, local):
     barrier(world)
     kv.sync_status()
     elapsed_ms = max_over_ranks(start.elapsed_time(stop), world, device)
-    launches = args.steps * (1 + 2 * BLOCKS)
+    launches = args.steps * (1 + BLOCKS)
 
     # ------------------------------------------------ per-launch attention time (roofline)
     # A second timed pass of the same steps with an event pair around every
@@ -255,7 +256,7 @@ def run_ours(args, world, rank, local):
         "tflops_per_step": round(step_tflops, 1),
         "frac_of_bf16_peak_step": round(step_tflops / sustained, 4),
         "served_frames_per_s": round(value / 4, 3),
-        "roofline": {"kernel": "attend_kernel<64>", "bound": "tensor",
+        "roofline": {"kernel": "attend_kernel<64> (fused record write)", "bound": "tensor",
                      "achieved": round(achieved_tflops, 1), "peak": sustained, "unit": "TFLOP/s",
                      "frac": round(achieved_tflops / sustained, 4),
                      "peak_source": f"bf16_tflops_sustained ({src})",
@@ -309,8 +310,7 @@ def run_e2e(args, torch, wm, kv, t, rank, world, device, Qd, Kd, Vd):
         for b in range(BLOCKS):
             comp.wait_event(landed[b])
             comp.wait_event(copied[b])
-            wm.wm_write_record(kv.h, b, t, dk[b], dv[b], comp)
-            wm.wm_attend(kv.h, b, dq[b], do[b], comp)
+            wm.wm_write_attend(kv.h, b, t, dq[b], dk[b], dv[b], do[b], comp)
             used[b].record(comp)
             s_out.wait_event(used[b])
             with torch.cuda.stream(s_out):

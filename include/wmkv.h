@@ -97,6 +97,17 @@ WM_API int wm_write_record(wm_kvbuf* h, int block, int64_t t, const void* K, con
  * (else WM_ERR_STATE). */
 WM_API int wm_attend(wm_kvbuf* h, int block, const void* Q, void* O, wm_stream_t stream);
 
+/* wm_write_record followed by wm_attend for the same block and frame, in one
+ * launch where the head dimension allows (d = 64): the attention reads the
+ * keys before and after the record's slot from the buffer and the record
+ * itself from K/V (softmax attention does not depend on the order of the
+ * keys), while the same launch copies K/V into the slot.  Results and buffer
+ * contents are exactly those of the two separate calls.  Arguments and errors
+ * as for wm_write_record and wm_attend (Q, K, V, O device [R, heads, d] bf16;
+ * t must be the current frame). */
+WM_API int wm_write_attend(wm_kvbuf* h, int block, int64_t t, const void* Q, const void* K,
+                           const void* V, void* O, wm_stream_t stream);
+
 /* Introspection (host only, no device work). */
 WM_API int64_t wm_end(const wm_kvbuf* h);                 /* end(t) at the current frame; -1 before t=0 */
 WM_API int64_t wm_capacity(const wm_kvbuf* h);            /* C */

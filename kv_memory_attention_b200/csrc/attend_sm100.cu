@@ -87,7 +87,13 @@ struct Cfg {
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + TILE_BYTES;
   static constexpr int V_OFF = K_OFF + NK * TILE_BYTES;
-  static constexpr int BAR_OFF = V_OFF + NV * TILE_BYTES;
+  // staging buffer of the in-kernel record copy (d = 64 only: for d = 128 the
+  // rings use the shared memory and the record is copied by its own launch)
+  static constexpr bool COPY_IN_KERNEL = (D == 64);
+  static constexpr int COPY_CHUNK_BYTES = 16384;  // per staging buffer (K and V chunk)
+  static constexpr int COPY_STAGE_BYTES = COPY_IN_KERNEL ? 2 * COPY_CHUNK_BYTES : 0;
+  static constexpr int COPY_OFF = V_OFF + NV * TILE_BYTES;
+  static constexpr int BAR_OFF = COPY_OFF + COPY_STAGE_BYTES;
   // barrier indices
   static constexpr int B_Q = 0;
   static constexpr int B_KFULL = 1;
@@ -100,7 +106,8 @@ struct Cfg {
   static constexpr int B_ODONE = B_PFULL + 2;    // 2
   static constexpr int B_OFINAL = B_ODONE + 2;
   static constexpr int B_DRAIN = B_OFINAL + 1;   // 3: one per MMA issuer
-  static constexpr int NBAR = B_DRAIN + 3;
+  static constexpr int B_COPY = B_DRAIN + 3;     // 2: record copy staging loads (K, V)
+  static constexpr int NBAR = B_COPY + 2;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;   // [0] tmem base, [1] abort
   // m[2][BM], l[2][BM] for the final merge; they reuse the Q tile, which no
   // MMA reads any more once the last P.V has completed
@@ -138,17 +145,46 @@ constexpr int poly_pairs_per_8() {
   return WMKV_POLY_PAIRS_PER_8 >= 0 ? WMKV_POLY_PAIRS_PER_8 : (D == 64 ? 3 : 0);
 }
 
+// Keys come in up to MAX_SEGS segments, each with its own K and V tensor
+// maps (row extent = the segment's length, so the rows past its end are
+// zero-filled).  Softmax attention does not depend on the order of the keys,
+// so the fused write+attend call reads the rows before and after the current
+// record's slot from the buffer and the record itself from the caller.
+constexpr int MAX_SEGS = 3;
+
 struct AttendParams {
   CUtensorMap tm_q;
-  CUtensorMap tm_k;
-  CUtensorMap tm_v;
+  CUtensorMap tm_k[MAX_SEGS];
+  CUtensorMap tm_v[MAX_SEGS];
   __nv_bfloat16* o;
   int64_t lq;
-  int64_t lk;
+  int seg_tiles_end[MAX_SEGS];  // cumulative number of 128-key tiles
+  int seg_rows[MAX_SEGS];       // keys in each segment
+  int nseg;
   int heads;
   float scale_log2;  // log2(e) / sqrt(d)
   int* status;       // may be null
+  // optional copy of a record into its slot, spread over the CTAs (16-byte units)
+  const uint4* copy_src[2];
+  uint4* copy_dst[2];
+  int64_t copy_n16;
 };
+
+// Segment and row of key tile j, and how many of its 128 rows are keys.
+struct TileLoc {
+  int seg;
+  int row;
+  int valid;
+};
+__device__ __forceinline__ TileLoc tile_loc(const AttendParams& p, int j) {
+  int seg = 0;
+#pragma unroll
+  for (int k = 0; k < MAX_SEGS - 1; ++k) seg += (k < p.nseg - 1 && j >= p.seg_tiles_end[k]) ? 1 : 0;
+  const int first = seg ? p.seg_tiles_end[seg - 1] : 0;
+  const int row = (j - first) * BN;
+  const int left = p.seg_rows[seg] - row;
+  return {seg, row, left < BN ? left : BN};
+}
 
 __device__ __forceinline__ void record_timeout(int* status) {
   if (status) atomicExch(status, DEV_TIMEOUT);
@@ -193,7 +229,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
   const int lane = threadIdx.x % 32;
   const int q_tile = blockIdx.x;
   const int head = blockIdx.y;
-  const int nkv = static_cast<int>((p.lk + BN - 1) / BN);
+  const int nkv = p.seg_tiles_end[p.nseg - 1];
 
   pdl_launch_dependents();
   if (threadIdx.x == 0) {
@@ -216,6 +252,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
     // for d = 64; for d = 128 the single issuer commits twice)
     mbar_init(bar(C::B_OFINAL), 2);
     for (int i = 0; i < 3; ++i) mbar_init(bar(C::B_DRAIN + i), 1);
+    mbar_init(bar(C::B_COPY), 1);
+    mbar_init(bar(C::B_COPY + 1), 1);
     misc[1] = 0;
     fence_mbar_init();
   }
@@ -225,8 +263,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
   }
   if (warp == 8 && lane == 0) {
     tma_prefetch_desc(&p.tm_q);
-    tma_prefetch_desc(&p.tm_k);
-    tma_prefetch_desc(&p.tm_v);
+    for (int k = 0; k < p.nseg; ++k) {
+      tma_prefetch_desc(&p.tm_k[k]);
+      tma_prefetch_desc(&p.tm_v[k]);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -247,18 +287,53 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
       for (int s = 0; s < C::SUB; ++s)
         tma_load_3d(sbase + C::Q_OFF + s * C::SUB_BYTES, &p.tm_q, s * 64, head, q_tile * BM,
                     bar(C::B_Q));
+      // This CTA's share of the record (fused write + attend), K and V chunks
+      // staged through shared memory with bulk copies.  Nothing in this launch
+      // reads the slot (its keys come from the caller's record), so the copy
+      // overlaps the first tiles; it runs once the K/V rings have been filled,
+      // where the producer would otherwise wait for a free slot.
+      bool copied = !(C::COPY_IN_KERNEL && p.copy_n16 > 0);
+      auto copy_record = [&]() {
+        const int64_t G = int64_t(gridDim.x) * gridDim.y;
+        const int64_t c = int64_t(blockIdx.y) * gridDim.x + blockIdx.x;
+        const int64_t per = (p.copy_n16 + G - 1) / G;
+        const int64_t lo = c * per;
+        const int64_t hi = lo + per < p.copy_n16 ? lo + per : p.copy_n16;
+        constexpr int64_t CH = C::COPY_CHUNK_BYTES / 16;
+        uint32_t cph = 0;
+        for (int64_t u = lo; u < hi && !*abort_flag; u += CH) {
+          const uint32_t bytes = static_cast<uint32_t>((hi - u < CH ? hi - u : CH) * 16);
+          bulk_wait_read_all();
+          for (int t = 0; t < 2; ++t) {
+            mbar_expect_tx(bar(C::B_COPY + t), bytes);
+            bulk_load(sbase + C::COPY_OFF + t * C::COPY_CHUNK_BYTES, p.copy_src[t] + u, bytes,
+                      bar(C::B_COPY + t));
+          }
+          for (int t = 0; t < 2; ++t) {
+            if (!mbar_wait_bounded(bar(C::B_COPY + t), cph, abort_flag, WAIT_LIMIT_CYCLES)) break;
+            bulk_store(p.copy_dst[t] + u, sbase + C::COPY_OFF + t * C::COPY_CHUNK_BYTES, bytes);
+          }
+          bulk_commit();
+          cph ^= 1;
+        }
+      };
       // K tile i and V tile i - K_AHEAD per step; each waits for its own ring slot
       int k_issued = 0, v_issued = 0;
       for (int i = 0; i < nkv + C::K_AHEAD; ++i) {
+        if (!copied && (i >= C::NK || i >= nkv)) {
+          copy_record();
+          copied = true;
+        }
         if (i < nkv) {
           const int st = i % C::NK;
           if (i >= C::NK && !mbar_wait_bounded(bar(C::B_KEMPTY + st), ((i / C::NK) - 1) & 1,
                                                abort_flag, WAIT_LIMIT_CYCLES))
             break;
+          const TileLoc tl = tile_loc(p, i);
           mbar_expect_tx(bar(C::B_KFULL + st), C::TILE_BYTES);
           for (int s = 0; s < C::SUB; ++s)
-            tma_load_3d(sbase + C::K_OFF + st * C::TILE_BYTES + s * C::SUB_BYTES, &p.tm_k, s * 64,
-                        head, i * BN, bar(C::B_KFULL + st));
+            tma_load_3d(sbase + C::K_OFF + st * C::TILE_BYTES + s * C::SUB_BYTES, &p.tm_k[tl.seg],
+                        s * 64, head, tl.row, bar(C::B_KFULL + st));
           k_issued = i + 1;
         }
         const int jv = i - C::K_AHEAD;
@@ -267,13 +342,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
           if (jv >= C::NV && !mbar_wait_bounded(bar(C::B_VEMPTY + st), ((jv / C::NV) - 1) & 1,
                                                 abort_flag, WAIT_LIMIT_CYCLES))
             break;
+          const TileLoc tl = tile_loc(p, jv);
           mbar_expect_tx(bar(C::B_VFULL + st), C::TILE_BYTES);
           for (int s = 0; s < C::SUB; ++s)
-            tma_load_3d(sbase + C::V_OFF + st * C::TILE_BYTES + s * C::SUB_BYTES, &p.tm_v, s * 64,
-                        head, jv * BN, bar(C::B_VFULL + st));
+            tma_load_3d(sbase + C::V_OFF + st * C::TILE_BYTES + s * C::SUB_BYTES, &p.tm_v[tl.seg],
+                        s * 64, head, tl.row, bar(C::B_VFULL + st));
           v_issued = jv + 1;
         }
       }
+      if (!copied) copy_record();
+      bulk_wait_all();   // bulk stores complete (no-op if none were issued)
       if (*abort_flag) {
         // Let the copies this thread started land before the CTA exits.
         volatile int no_abort = 0;
@@ -437,8 +515,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
       float s[128];
 #pragma unroll
       for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
-      if (j == nkv - 1) {
-        const int valid = static_cast<int>(p.lk - int64_t(j) * BN);
+      {
+        const int valid = tile_loc(p, j).valid;
         if (valid < BN) {
 #pragma unroll
           for (int c = 0; c < 128; ++c)
@@ -640,18 +718,38 @@ cudaError_t launch_d(const AttendParams& prm, int64_t lq, int heads, cudaStream_
 
 }  // namespace
 
-cudaError_t launch_attend(const void* q, const void* k, const void* v, void* o, int64_t lq,
-                          int64_t lk, int heads, int d, int* status, cudaStream_t stream) {
-  AttendParams prm;
-  if (!encode_rows_map(&prm.tm_q, q, lq, heads, d) || !encode_rows_map(&prm.tm_k, k, lk, heads, d) ||
-      !encode_rows_map(&prm.tm_v, v, lk, heads, d))
-    return cudaErrorInvalidValue;
+bool attend_copies_in_kernel(int d) { return Cfg<64>::COPY_IN_KERNEL && d == 64; }
+
+cudaError_t launch_attend(const void* q, void* o, int64_t lq, const KVSegment* segs, int nseg,
+                          int heads, int d, int* status, const RecordCopy* copy,
+                          cudaStream_t stream) {
+  if (nseg < 1 || nseg > MAX_SEGS) return cudaErrorInvalidValue;
+  AttendParams prm = {};
+  if (!encode_rows_map(&prm.tm_q, q, lq, heads, d)) return cudaErrorInvalidValue;
+  int tiles = 0;
+  for (int k = 0; k < nseg; ++k) {
+    if (segs[k].rows < 1 || segs[k].rows >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
+    if (!encode_rows_map(&prm.tm_k[k], segs[k].k, segs[k].rows, heads, d) ||
+        !encode_rows_map(&prm.tm_v[k], segs[k].v, segs[k].rows, heads, d))
+      return cudaErrorInvalidValue;
+    tiles += static_cast<int>((segs[k].rows + BN - 1) / BN);
+    prm.seg_tiles_end[k] = tiles;
+    prm.seg_rows[k] = static_cast<int>(segs[k].rows);
+  }
+  prm.nseg = nseg;
   prm.o = static_cast<__nv_bfloat16*>(o);
   prm.lq = lq;
-  prm.lk = lk;
   prm.heads = heads;
   prm.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
   prm.status = status;
+  if (copy && copy->n16 > 0) {
+    if (!attend_copies_in_kernel(d)) return cudaErrorInvalidValue;
+    prm.copy_src[0] = static_cast<const uint4*>(copy->k_src);
+    prm.copy_src[1] = static_cast<const uint4*>(copy->v_src);
+    prm.copy_dst[0] = static_cast<uint4*>(copy->k_dst);
+    prm.copy_dst[1] = static_cast<uint4*>(copy->v_dst);
+    prm.copy_n16 = copy->n16;
+  }
   if (d == 64) return launch_d<64>(prm, lq, heads, stream);
   if (d == 128) return launch_d<128>(prm, lq, heads, stream);
   return cudaErrorInvalidValue;

@@ -192,9 +192,48 @@ int wm_attend(wm_kvbuf* h, int block, const void* Q, void* O, wm_stream_t stream
   const int64_t end = end_at(h->HW, h->X, h->Y, h->W, h->t);
   const uint8_t* kbuf = h->buf + int64_t(block) * h->block_bytes;
   const uint8_t* vbuf = kbuf + h->tensor_bytes;
-  cudaError_t e = wmkv::launch_attend(Q, kbuf, vbuf, O, h->R, end, h->heads, h->d, h->status,
+  const wmkv::KVSegment seg = {kbuf, vbuf, end};
+  cudaError_t e = wmkv::launch_attend(Q, O, h->R, &seg, 1, h->heads, h->d, h->status, nullptr,
                                       reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
+  return WM_OK;
+}
+
+int wm_write_attend(wm_kvbuf* h, int block, int64_t t, const void* Q, const void* K,
+                    const void* V, void* O, wm_stream_t stream) {
+  if (!h || block < 0 || block >= h->blocks || !aligned16(Q) || !aligned16(K) || !aligned16(V) ||
+      !aligned16(O))
+    return WM_ERR_INVALID_ARG;
+  if (h->t < 0 || t != h->t) return WM_ERR_STATE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t row0 = record_row(h->HW, h->X, h->Y, t);
+  uint8_t* kbuf = h->buf + int64_t(block) * h->block_bytes;
+  uint8_t* vbuf = kbuf + h->tensor_bytes;
+  uint8_t* kslot = kbuf + row0 * h->row_bytes;
+  uint8_t* vslot = vbuf + row0 * h->row_bytes;
+  const int64_t n16 = h->R * h->row_bytes / 16;
+  const int64_t end = end_at(h->HW, h->X, h->Y, h->W, t);
+  cudaError_t e;
+  if (wmkv::attend_copies_in_kernel(h->d)) {
+    // keys: buffer rows before the slot, buffer rows after it, and the record
+    // itself from the caller (the slot is being written by the same launch)
+    wmkv::KVSegment segs[3];
+    int nseg = 0;
+    if (row0 > 0) segs[nseg++] = {kbuf, vbuf, row0};
+    const int64_t after = row0 + h->R;
+    if (end > after)
+      segs[nseg++] = {kbuf + after * h->row_bytes, vbuf + after * h->row_bytes, end - after};
+    segs[nseg++] = {K, V, h->R};
+    const wmkv::RecordCopy cp = {K, V, kslot, vslot, n16};
+    e = wmkv::launch_attend(Q, O, h->R, segs, nseg, h->heads, h->d, h->status, &cp, s);
+  } else {
+    e = wmkv::launch_copy_pair(K, V, kslot, vslot, n16, s);
+    const wmkv::KVSegment seg = {kbuf, vbuf, end};
+    if (e == cudaSuccess)
+      e = wmkv::launch_attend(Q, O, h->R, &seg, 1, h->heads, h->d, h->status, nullptr, s);
+  }
+  if (e != cudaSuccess) return cuda_fail(e);
+  h->written[block] = t;
   return WM_OK;
 }
 
@@ -269,7 +308,8 @@ int wm_attend_dense(const void* Q, const void* K, const void* V, void* O, int64_
     return WM_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return WM_ERR_UNSUPPORTED;
   if ((Lq + 127) / 128 > 0x7FFFFFFF || heads > 65535) return WM_ERR_INVALID_ARG;
-  cudaError_t e = wmkv::launch_attend(Q, K, V, O, Lq, Lk, heads, d, dev_status,
+  const wmkv::KVSegment seg = {K, V, Lk};
+  cudaError_t e = wmkv::launch_attend(Q, O, Lq, &seg, 1, heads, d, dev_status, nullptr,
                                       reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
   return WM_OK;

@@ -35,11 +35,31 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 constexpr int DEV_OK = 0;
 constexpr int DEV_TIMEOUT = 1;
 
-// Dense flash attention over keys [0, lk): see attend_sm100.cu.
-// Q/O: [lq, heads, d]; K/V: rows [0, lk) of arrays whose rows are `heads*d`
-// bf16 values.  Returns a cudaError_t from encoding/launching.
-cudaError_t launch_attend(const void* q, const void* k, const void* v, void* o, int64_t lq,
-                          int64_t lk, int heads, int d, int* status, cudaStream_t stream);
+// A run of keys: rows [0, rows) of K and V arrays whose rows are `heads*d`
+// bf16 values.
+struct KVSegment {
+  const void* k;
+  const void* v;
+  int64_t rows;
+};
+// A record copy the attention launch performs on the side (K and V, n16
+// 16-byte units each).
+struct RecordCopy {
+  const void* k_src;
+  const void* v_src;
+  void* k_dst;
+  void* v_dst;
+  int64_t n16;
+};
+
+// Dense flash attention of Q [lq, heads, d] over the keys of 1..3 segments
+// (softmax over all of them together), O [lq, heads, d]: see attend_sm100.cu.
+// `copy` (may be null) is performed by the same launch; only supported where
+// attend_copies_in_kernel(d).  Returns a cudaError_t from encoding/launching.
+cudaError_t launch_attend(const void* q, void* o, int64_t lq, const KVSegment* segs, int nseg,
+                          int heads, int d, int* status, const RecordCopy* copy,
+                          cudaStream_t stream);
+bool attend_copies_in_kernel(int d);
 
 // Copy `n16` 16-byte chunks of a and b (two independent arrays) in one launch.
 cudaError_t launch_copy_pair(const void* a_src, const void* b_src, void* a_dst, void* b_dst,

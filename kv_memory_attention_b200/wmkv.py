@@ -31,6 +31,7 @@ SIGNATURES = {
     "wm_advance": (_c_int, [_vp, _c_i64, _vp]),
     "wm_write_record": (_c_int, [_vp, _c_int, _c_i64, _vp, _vp, _vp]),
     "wm_attend": (_c_int, [_vp, _c_int, _vp, _vp, _vp]),
+    "wm_write_attend": (_c_int, [_vp, _c_int, _c_i64, _vp, _vp, _vp, _vp, _vp]),
     "wm_end": (_c_i64, [_vp]),
     "wm_capacity": (_c_i64, [_vp]),
     "wm_current_frame": (_c_i64, [_vp]),
@@ -121,6 +122,11 @@ def wm_write_record(h: int, block: int, t: int, K, V, stream=None) -> None:
 
 def wm_attend(h: int, block: int, Q, O, stream=None) -> None:
     _check(LIB.wm_attend(h, block, _ptr(Q), _ptr(O), _stream(stream)), "wm_attend")
+
+
+def wm_write_attend(h: int, block: int, t: int, Q, K, V, O, stream=None) -> None:
+    _check(LIB.wm_write_attend(h, block, t, _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _stream(stream)),
+           "wm_write_attend")
 
 
 def wm_end(h: int) -> int:
@@ -220,6 +226,9 @@ class KVMemory:
 
     def attend(self, block, Q, O, stream=None):
         wm_attend(self.h, block, Q, O, stream)
+
+    def write_attend(self, block, t, Q, K, V, O, stream=None):
+        wm_write_attend(self.h, block, t, Q, K, V, O, stream)
 
     def end(self):
         return wm_end(self.h)

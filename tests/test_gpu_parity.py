@@ -179,3 +179,62 @@ def test_wide_score_range_exercises_rescaling(wm, d):
 def test_sampled_rows_helper_is_in_range():
     rows = sample_rows(SERVED, 0)
     assert rows.min() == 0 and rows.max() == SERVED.R - 1 and len(rows) >= 60
+
+
+# ------------------------------------------------------------ fused write + attend
+
+@pytest.mark.parametrize("L,frames", [
+    (TINY, range(12)),
+    (Layout(24, 42, 96, 2, 24, heads=4, d=64), range(30)),
+    (Layout(3, 5, 2, 0, 4, heads=2, d=64), range(9)),
+    (Layout(5, 7, 9, 2, 9, heads=2, d=128), range(14)),
+])
+def test_write_attend_equals_write_then_attend(wm, L, frames):
+    """One launch (keys: buffer before/after the slot + the record from the caller) gives
+    the same buffer bytes as write_record followed by attend, and the same attention."""
+    blocks = 2
+    a = wm.KVMemory(blocks, L.heads, L.d, L.grid_h, L.grid_w, L.X, L.Y, L.W)
+    b = wm.KVMemory(blocks, L.heads, L.d, L.grid_h, L.grid_w, L.X, L.Y, L.W)
+    mem = FrameMemory(L, blocks, track_records=False)
+    for t in frames:
+        a.advance(t)
+        b.advance(t)
+        mem.advance(t)
+        for step in range(2):
+            for blk in range(blocks):
+                q, k, v = si.record_inputs(21, 0, blk, t, step, L.R, L.heads, L.d)
+                qd, kd, vd = dev(q), dev(k), dev(v)
+                oa, ob = nan_like((L.R, L.heads, L.d)), nan_like((L.R, L.heads, L.d))
+                a.write_record(blk, t, kd, vd)
+                a.attend(blk, qd, oa)
+                b.write_attend(blk, t, qd, kd, vd, ob)
+                mem.write_record(blk, t, k, v)
+                ref = attend_memory(mem, blk, q)
+                assert_attn_close(host_bits(oa), ref, f"separate t={t}")
+                assert_attn_close(host_bits(ob), ref, f"fused t={t}")
+        torch.cuda.synchronize()
+        for blk in range(blocks):
+            ka, va = a.kv_views(blk)
+            kb, vb = b.kv_views(blk)
+            assert torch.equal(ka, kb) and torch.equal(va, vb), f"buffers differ at t={t}"
+            assert np.array_equal(host_bits(kb), mem.K[blk]) and np.array_equal(host_bits(vb), mem.V[blk])
+    a.sync_status()
+    b.sync_status()
+
+
+def test_write_attend_state_errors(wm):
+    L = TINY
+    kv = wm.KVMemory(1, L.heads, L.d, L.grid_h, L.grid_w, L.X, L.Y, L.W)
+    q = torch.zeros(L.R, L.heads, L.d, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(wm.WmError) as e:
+        kv.write_attend(0, 0, q, q, q, q)          # before advance(0)
+    assert e.value.code == wm.WM_ERR_STATE
+    kv.advance(0)
+    with pytest.raises(wm.WmError) as e:
+        kv.write_attend(0, 1, q, q, q, q)          # wrong frame
+    assert e.value.code == wm.WM_ERR_STATE
+    with pytest.raises(wm.WmError) as e:
+        kv.write_attend(1, 0, q, q, q, q)          # no such block
+    assert e.value.code == wm.WM_ERR_INVALID_ARG
+    kv.write_attend(0, 0, q, q, q, q)
+    kv.sync_status()

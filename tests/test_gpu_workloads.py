@@ -2,7 +2,7 @@
 
 * full rollout: 28 blocks at the served shape, frames 0..40 from an empty
   buffer, 4 passes (write + attend) per frame, inputs seeded per
-  (block, frame, pass);
+  (block, frame, pass); half of the passes use the fused wm_write_attend;
 * batch of 8 independent sessions (28 blocks each) in steady state, K rows
   scaled by U(0.5, 2) per token;
 * scaled memory: 45x80 grid + 256 summary tokens, Y=2, W=48, 24 heads x 128,
@@ -61,13 +61,16 @@ def test_full_rollout_28_blocks_four_passes(wm, pool):
                 sk = si.seed_for(3, 0, b, t, step, si.T_K)
                 sv = si.seed_for(3, 0, b, t, step, si.T_V)
                 kd, vd = pool.normal(sk, shape), pool.normal(sv, shape)
-                kv.write_record(b, t, kd, vd)
+                sq = si.seed_for(3, 0, b, t, step, si.T_Q)
+                o = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+                if (step + b) % 2:                 # fused call on half of the passes
+                    kv.write_attend(b, t, pool.normal(sq, shape), kd, vd, o)
+                else:
+                    kv.write_record(b, t, kd, vd)
+                    kv.attend(b, pool.normal(sq, shape), o)
                 mem.write_record(b, t, si.pool_normal_bf16(sk, shape), si.pool_normal_bf16(sv, shape))
                 kb, vb = kv.kv_views(b)
                 assert torch.equal(kb[r0:r1], kd) and torch.equal(vb[r0:r1], vd), (t, step, b)
-                sq = si.seed_for(3, 0, b, t, step, si.T_Q)
-                o = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
-                kv.attend(b, pool.normal(sq, shape), o)
                 if b in SAMPLED_BLOCKS:
                     rows = sample_rows(L, hash((t, step, b)) & 0xFFFF)
                     ref = attend_memory(mem, b, si.pool_normal_bf16(sq, shape), rows=rows)
