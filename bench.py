@@ -132,7 +132,8 @@ def init_pg(world, backend):
     return dist
 
 
-def max_over_ranks(x: float, world: int, device) -> float:
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Largest value over all ranks (the slowest rank sets the job's time)."""
     if world == 1:
         return x
     import torch
@@ -140,6 +141,11 @@ def max_over_ranks(x: float, world: int, device) -> float:
     t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_throughput(steps_per_rank: int, elapsed_ms_max: float, world: int) -> float:
+    """Whole-job frame-steps/s: all ranks' steps over the slowest rank's time."""
+    return world * steps_per_rank / (elapsed_ms_max / 1e3)
 
 
 def barrier(world):
@@ -238,7 +244,7 @@ def run_ours(args, world, rank, local):
     t = e2e.pop("_t")
     kv.sync_status()
 
-    value = world * args.steps / (elapsed_ms / 1e3)
+    value = aggregate_throughput(args.steps, elapsed_ms, world)
     sustained, burst, hbm, src = peaks()
     achieved_tflops = ATTN_FLOP / (attn_avg_ms * 1e-3) / 1e12
     step_tflops = BLOCKS * ATTN_FLOP * args.steps / (elapsed_ms / 1e3) / 1e12
