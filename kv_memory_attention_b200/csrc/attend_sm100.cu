@@ -140,6 +140,13 @@ struct Cfg {
 #ifndef WMKV_POLY_PAIRS_PER_8
 #define WMKV_POLY_PAIRS_PER_8 -1
 #endif
+// Exponentials two per MUFU instruction in f16 (argument and result), widened
+// to f32 for the row sum and packed to bf16 for P.V.
+#ifndef WMKV_EXP_F16X2
+#define WMKV_EXP_F16X2 0
+#endif
+constexpr bool EXP_F16X2 = WMKV_EXP_F16X2 != 0;
+
 template <int D>
 constexpr int poly_pairs_per_8() {
   return WMKV_POLY_PAIRS_PER_8 >= 0 ? WMKV_POLY_PAIRS_PER_8 : (D == 64 ? 3 : 0);
@@ -553,7 +560,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
       for (int pp = 0; pp < 64; ++pp) {
         const f2 x = f2_fma(f2_make(s[2 * pp], s[2 * pp + 1]), scale2, negm2);
         f2 e;
-        if ((pp % 8) >= 8 - poly_pairs_per_8<D>()) {
+        if (EXP_F16X2) {
+          e = exp2_f16x2(x);
+        } else if ((pp % 8) >= 8 - poly_pairs_per_8<D>()) {
           e = exp2_poly2(x);
         } else {
           float x0, x1;

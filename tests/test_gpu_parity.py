@@ -82,6 +82,27 @@ def test_small_geometries(wm, L):
     roll(wm, L, 2, range(2 * L.W + 3), 2, config_id=12)
 
 
+def test_served_default_window_w16(wm):
+    """The server's default window W = 16 (C = 5,760 keys): rolled to steady state, all rows of
+    one block checked at t = 17..19 through the fused call."""
+    L = Layout(24, 42, 96, 2, 16, heads=16, d=64)
+    assert L.C == 4 * L.R + 14 * 96 == 5760
+    kv = wm.KVMemory(1, L.heads, L.d, L.grid_h, L.grid_w, L.X, L.Y, L.W)
+    mem = FrameMemory(L, 1, track_records=False)
+    for t in range(20):
+        kv.advance(t)
+        mem.advance(t)
+        q, k, v = si.record_inputs(6, 0, 0, t, 0, L.R, L.heads, L.d)
+        o = nan_like((L.R, L.heads, L.d))
+        kv.write_attend(0, t, dev(q), dev(k), dev(v), o)
+        mem.write_record(0, t, k, v)
+        check_buffers(kv, mem)
+        if t >= 17:
+            assert kv.end() == 5760
+            assert_attn_close(host_bits(o), attend_memory(mem, 0, q), f"W=16 t={t}")
+    kv.sync_status()
+
+
 def test_served_single_block_steady_state(wm):
     """Served shape, one block rolled write-only to t=31; attend with all 1104 queries over 6,528 keys."""
     L = SERVED
