@@ -8,8 +8,10 @@ library.
 """
 from .kvmemory import (Layout, FrameMemory, attend, attend_bits, attend_memory,
                        softmax_weights, visible_history_mask, masked_history_attend,
+                       rotation_cos_sin, rotate_pairs_f64, rotate_keys_bf16, sink_shift,
                        TINY, SERVED, SERVED_W16, SCALED)
 
 __all__ = ["Layout", "FrameMemory", "attend", "attend_bits", "attend_memory",
            "softmax_weights", "visible_history_mask", "masked_history_attend",
+           "rotation_cos_sin", "rotate_pairs_f64", "rotate_keys_bf16", "sink_shift",
            "TINY", "SERVED", "SERVED_W16", "SCALED"]

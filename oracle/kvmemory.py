@@ -41,6 +41,18 @@ notes of the repository):
   R5 attention uses scale 1/sqrt(d) and an ordinary softmax (the page names
      the attention kernels, FlexAttention and flash_attn_with_kvcache, whose
      default is this scale).
+  R6 (section "Running for a long time: the start image follows the window")
+     the oldest frame in memory while frame t is generated is max(1, t - W);
+     the gap is that frame's id minus the start image's temporal position,
+     which starts at 0.  When the gap reaches 5 at the start of a frame, the
+     start image's keys (Z0 rows of K, every block) are rotated forward by
+     gap - 1 frames, in place; values are untouched.  The rotation acts on
+     adjacent dimension pairs (2i, 2i+1) of each head as on complex numbers,
+     pair i turning by theta_i * shift (theta_i = 0: not a temporal pair),
+     computed in float32 as a' = a*c - b*s, b' = a*s + b*c (each product and
+     sum rounded to float32, c and s the float32 cosine and sine) and rounded
+     to bfloat16: the page gives neither the frequencies nor the precision,
+     so the frequencies are a parameter and the precision is the kernel's.
 """
 from __future__ import annotations
 
@@ -133,6 +145,56 @@ class Layout:
 
 
 # ---------------------------------------------------------------------------
+# Streaming sink: section "Running for a long time" (reading R6)
+# ---------------------------------------------------------------------------
+
+def rotation_cos_sin(theta, shift: int):
+    """float32 cosine and sine of theta_i * shift (double precision, then rounded)."""
+    ang = np.asarray(theta, dtype=np.float64) * float(shift)
+    return np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
+
+
+def rotate_pairs_f64(x: np.ndarray, theta, shift: float) -> np.ndarray:
+    """Exact-arithmetic reference: adjacent pairs of the last axis turned by theta_i * shift."""
+    x = np.asarray(x, dtype=np.float64)
+    ang = np.asarray(theta, dtype=np.float64) * shift
+    a, b = x[..., 0::2], x[..., 1::2]
+    out = np.empty_like(x)
+    out[..., 0::2] = a * np.cos(ang) - b * np.sin(ang)
+    out[..., 1::2] = a * np.sin(ang) + b * np.cos(ang)
+    return out
+
+
+def rotate_keys_bf16(k_bits: np.ndarray, theta, shift: int) -> np.ndarray:
+    """The in-place key rotation as stored: float32 arithmetic in a fixed order, then bf16.
+
+    Pairs with theta_i == 0 are left untouched (bit for bit).
+    """
+    c, s = rotation_cos_sin(theta, shift)
+    x = si.bf16_bits_to_f32(k_bits)
+    a, b = x[..., 0::2], x[..., 1::2]
+    na = np.subtract(np.multiply(a, c, dtype=np.float32), np.multiply(b, s, dtype=np.float32),
+                     dtype=np.float32)
+    nb = np.add(np.multiply(a, s, dtype=np.float32), np.multiply(b, c, dtype=np.float32),
+                dtype=np.float32)
+    out = np.array(k_bits, dtype=np.uint16, copy=True)
+    rot = np.asarray(theta) != 0
+    ra, rb = si.f32_to_bf16_bits(na), si.f32_to_bf16_bits(nb)
+    out[..., 0::2] = np.where(rot, ra, out[..., 0::2])
+    out[..., 1::2] = np.where(rot, rb, out[..., 1::2])
+    return out
+
+
+def sink_shift(layout: "Layout", t: int, z0_pos: int, trigger: int = 5, target: int = 1) -> int:
+    """Frames to move the start image forward at the start of frame t (0: no rotation)."""
+    if t < 1:
+        return 0
+    oldest = max(1, t - layout.W)
+    gap = oldest - z0_pos
+    return gap - target if gap >= trigger else 0
+
+
+# ---------------------------------------------------------------------------
 # The memory: a host mirror updated by the page's rules
 # ---------------------------------------------------------------------------
 
@@ -151,6 +213,8 @@ class FrameMemory:
     K: np.ndarray = field(init=False)
     V: np.ndarray = field(init=False)
     records: dict = field(init=False)       # (block, frame) -> (K rows, V rows)
+    sink_theta: object = None                # per-pair temporal frequencies (None: no sink)
+    z0_pos: int = 0                          # temporal position of the start image
     raw_tag: list = field(init=False)        # frame id held by each RAW slot
     sum_tag: list = field(init=False)        # frame id whose summary each SUM slot holds
     written: set = field(init=False)         # blocks written at the current t
@@ -186,6 +250,15 @@ class FrameMemory:
             self.K[:, d0:d1] = self.K[:, src0:r1]
             self.V[:, d0:d1] = self.V[:, src0:r1]
             self.sum_tag[u] = f
+        if self.sink_theta is not None:
+            shift = sink_shift(L, t, self.z0_pos)
+            if shift:
+                self.K[:, :L.R] = rotate_keys_bf16(self.K[:, :L.R], self.sink_theta, shift)
+                if self.track_records:
+                    for (b, f), (kf, vf) in list(self.records.items()):
+                        if f == 0:
+                            self.records[(b, 0)] = (self.K[b, :L.R].copy(), vf)
+                self.z0_pos += shift
         self.t = t
         self.written = set()
 

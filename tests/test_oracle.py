@@ -268,3 +268,97 @@ def test_bf16_rounding_is_nearest_even():
     x = np.array([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -(1.0 + 2.0 ** -8)], np.float32)
     out = si.bf16_bits_to_f64(si.f32_to_bf16_bits(x))
     assert out[0] == 1.0 and out[1] == 1.0 + 2.0 ** -6 and out[2] == -1.0
+
+
+# ---------------------------------------------------- streaming sink (start image keys)
+
+from oracle import rotate_keys_bf16, rotate_pairs_f64, rotation_cos_sin, sink_shift
+
+THETA = np.array([1.0e-4 * 10000.0 ** (-i / 16) for i in range(32)])   # 32 pairs of d = 64
+THETA[12:] = 0.0                                                        # 12 temporal pairs
+
+
+def test_rotation_composes_as_the_page_states():
+    """rotation(id + T) = rotation(id) * rotation(T)."""
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((5, 3, 64))
+    th = rng.uniform(0, 2, 32)
+    two = rotate_pairs_f64(rotate_pairs_f64(x, th, 7.0), th, 13.0)
+    np.testing.assert_allclose(two, rotate_pairs_f64(x, th, 20.0), rtol=0, atol=1e-12)
+
+
+def test_joint_rotation_keeps_scores_and_only_relative_shift_matters():
+    rng = np.random.default_rng(12)
+    q, k = rng.standard_normal((4, 64)), rng.standard_normal((9, 64))
+    th = rng.uniform(0, 1, 32)
+    s0 = q @ k.T
+    np.testing.assert_allclose(rotate_pairs_f64(q, th, 5.0) @ rotate_pairs_f64(k, th, 5.0).T, s0,
+                               rtol=0, atol=1e-12)
+    a = rotate_pairs_f64(q, th, 11.0) @ rotate_pairs_f64(k, th, 4.0).T
+    b = rotate_pairs_f64(q, th, 7.0) @ k.T
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+    # and it is not the identity: a shift of the keys alone changes the scores
+    assert np.abs(q @ rotate_pairs_f64(k, th, 3.0).T - s0).max() > 1e-3
+
+
+def test_rotation_keeps_pair_norms_and_quarter_turn():
+    rng = np.random.default_rng(13)
+    x = rng.standard_normal((6, 64))
+    th = rng.uniform(0, 3, 32)
+    y = rotate_pairs_f64(x, th, 2.0)
+    np.testing.assert_allclose(x[:, 0::2] ** 2 + x[:, 1::2] ** 2, y[:, 0::2] ** 2 + y[:, 1::2] ** 2,
+                               rtol=1e-12)
+    q = rotate_pairs_f64(x, np.full(32, np.pi / 2), 1.0)           # (a, b) -> (-b, a)
+    np.testing.assert_allclose(q[:, 0::2], -x[:, 1::2], atol=1e-12)
+    np.testing.assert_allclose(q[:, 1::2], x[:, 0::2], atol=1e-12)
+
+
+def test_stored_rotation_identity_cases_and_rounding():
+    k = si.normal_bf16(99, (7, 2, 64))
+    assert np.array_equal(rotate_keys_bf16(k, THETA, 0), k)          # shift 0: cos 1, sin 0
+    out = rotate_keys_bf16(k, THETA, 9)
+    assert np.array_equal(out[..., 24:], k[..., 24:])                 # non-temporal pairs untouched
+    exact = rotate_pairs_f64(si.bf16_bits_to_f64(k), THETA, 9.0)
+    got = si.bf16_bits_to_f64(out)
+    assert np.all(np.abs(got - exact) <= 2.0 ** -8 * np.abs(exact) + 1e-30 + 2.0 ** -120)
+    c, s = rotation_cos_sin(THETA, 9)
+    assert c.dtype == np.float32 and np.all(c[12:] == 1) and np.all(s[12:] == 0)
+
+
+@pytest.mark.parametrize("layout", [SERVED, TINY, SERVED_W16])
+def test_sink_schedule_keeps_gap_between_one_and_four(layout):
+    """The gap to the oldest frame in memory reaches 5 and is brought back to 1."""
+    z0, rotations = 0, []
+    for t in range(0, 200):
+        shift = sink_shift(layout, t, z0)
+        oldest = max(1, t - layout.W) if t >= 1 else None
+        if shift:
+            assert oldest - z0 == 5 and shift == 4
+            rotations.append(t)
+            z0 += shift
+        if t >= 1:
+            assert 1 <= oldest - z0 <= 4
+    first = layout.W + 5
+    assert rotations[0] == first and all(b - a == 4 for a, b in zip(rotations, rotations[1:]))
+
+
+def test_memory_rotates_only_start_image_keys():
+    L = Layout(2, 3, 2, 1, 3, heads=2, d=64)
+    mem = FrameMemory(L, blocks=2)
+    mem.sink_theta = THETA
+    prev_pos = 0
+    for t in range(12):
+        before = mem.K.copy(), mem.V.copy()
+        mem.advance(t)
+        shift_happened = mem.z0_pos != prev_pos
+        if shift_happened:
+            assert not np.array_equal(mem.K[:, :L.R], before[0][:, :L.R])
+        else:
+            assert np.array_equal(mem.K[:, :L.R], before[0][:, :L.R])
+        assert np.array_equal(mem.V[:, :L.R], before[1][:, :L.R])        # values untouched
+        prev_pos = mem.z0_pos
+        for b in range(2):
+            _, k, v = si.record_inputs(31, 0, b, t, 0, L.R, L.heads, L.d)
+            mem.write_record(b, t, k, v)
+        mem.check_against_records()
+    assert mem.z0_pos == 4              # one rotation, at t = W + 5 = 8 (the next would be t = 12)
