@@ -108,6 +108,27 @@ WM_API int wm_attend(wm_kvbuf* h, int block, const void* Q, void* O, wm_stream_t
 WM_API int wm_write_attend(wm_kvbuf* h, int block, int64_t t, const void* Q, const void* K,
                            const void* V, void* O, wm_stream_t stream);
 
+/* Streaming sink (model card section "Running for a long time: the start
+ * image follows the window"): frame ids keep growing while the start image
+ * was written at id 0; whenever the gap between the start image's temporal
+ * position and the oldest frame in memory (max(1, t-W) while frame t is
+ * generated) reaches `gap_trigger` (the page: 5), wm_advance(t) rotates the
+ * start image's keys (Z0 rows of K, every block) forward in place by
+ * gap - gap_target frames (the page: back to a gap of 1).  Values are not
+ * touched.  The page gives no rotary frequencies, so the caller passes them:
+ * theta[i] (radians per frame, host array of n_pairs = d/2 floats) for the
+ * adjacent dimension pair (2i, 2i+1) of every head, 0 for pairs outside the
+ * temporal band.  Pair i turns as a complex number by theta[i]*shift, in
+ * float32 (each product and sum rounded separately) then rounded to bf16.
+ * Must be called before the first wm_advance (else WM_ERR_STATE). */
+WM_API int wm_set_sink(wm_kvbuf* h, const float* theta, int n_pairs, int gap_trigger,
+                       int gap_target);
+/* Temporal position of the start image's keys (0 until the first rotation). */
+WM_API int64_t wm_sink_position(const wm_kvbuf* h);
+/* The float32 cosines and sines a rotation by `shift` frames uses (host
+ * arrays of d/2 floats). */
+WM_API int wm_sink_cos_sin(const wm_kvbuf* h, int64_t shift, float* c, float* s);
+
 /* Introspection (host only, no device work). */
 WM_API int64_t wm_end(const wm_kvbuf* h);                 /* end(t) at the current frame; -1 before t=0 */
 WM_API int64_t wm_capacity(const wm_kvbuf* h);            /* C */

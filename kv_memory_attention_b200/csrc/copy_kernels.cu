@@ -9,6 +9,7 @@
 // Both are contiguous copies in the token-major buffer layout, moved as
 // 16-byte vectors with several independent loads in flight per thread and a
 // grid sized to the SM count.
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "sm100_ptx.cuh"
@@ -73,6 +74,43 @@ __global__ void __launch_bounds__(COPY_THREADS) evict_kernel(uint8_t* base, int6
   copy_span(src, dst, n, int64_t(blockIdx.x) * COPY_THREADS + threadIdx.x, stride);
 }
 
+// Start image keys moved forward in time (model card "GTA world model:
+// weights and inference code", section "Running for a long time: the start
+// image follows the window"): RoPE keys are rotations, so multiplying a stored
+// key by one more rotation moves it forward; only the keys of the start
+// image (Z0 rows of every block's K buffer) change, in place.
+// Adjacent dimension pairs (2i, 2i+1) of each head turn by (c_i, s_i) as
+// complex numbers, in float32 with every product and sum rounded separately
+// (no fused multiply-add), then to bf16; pairs whose bit in `mask` is clear
+// are left untouched.  One thread per 16-byte vector (4 pairs).
+__global__ void __launch_bounds__(COPY_THREADS) rotate_z0_kernel(uint8_t* base, int64_t block_stride,
+                                                                 int64_t vec_per_block,
+                                                                 int vec_per_row_head,
+                                                                 SinkTable tab) {
+  pdl_launch_dependents();
+  pdl_wait_prior();
+  const int64_t i = int64_t(blockIdx.x) * COPY_THREADS + threadIdx.x;
+  if (i >= vec_per_block) return;
+  uint4* v = reinterpret_cast<uint4*>(base + int64_t(blockIdx.y) * block_stride) + i;
+  const int pair0 = static_cast<int>(i % vec_per_row_head) * 4;
+  uint4 x = *v;
+  uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int pr = pair0 + k;
+    if (!((tab.mask >> pr) & 1ull)) continue;
+    const float a = __uint_as_float(w[k] << 16);
+    const float b = __uint_as_float(w[k] & 0xFFFF0000u);
+    const float c = tab.c[pr], s = tab.s[pr];
+    const float na = __fsub_rn(__fmul_rn(a, c), __fmul_rn(b, s));
+    const float nb = __fadd_rn(__fmul_rn(a, s), __fmul_rn(b, c));
+    const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(na));
+    const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(nb));
+    w[k] = lo | (hi << 16);
+  }
+  *v = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 int sm_count() {
   static int n = 0;
   if (n == 0) {
@@ -104,6 +142,18 @@ cudaError_t launch_copy_pair(const void* a_src, const void* b_src, void* a_dst, 
   return launch_pdl(copy_pair_kernel, grid, dim3(COPY_THREADS), 0, stream,
                     static_cast<const uint4*>(a_src), static_cast<const uint4*>(b_src),
                     static_cast<uint4*>(a_dst), static_cast<uint4*>(b_dst), n16);
+}
+
+cudaError_t launch_rotate_z0(void* base, int blocks, int64_t block_stride_bytes, int64_t rows,
+                             int heads, int d, const SinkTable& tab, cudaStream_t stream) {
+  const int64_t vec_per_row_head = d / 8;
+  const int64_t vec_per_block = rows * heads * vec_per_row_head;
+  if (vec_per_block <= 0 || blocks <= 0) return cudaSuccess;
+  dim3 grid(static_cast<unsigned>((vec_per_block + COPY_THREADS - 1) / COPY_THREADS),
+            static_cast<unsigned>(blocks));
+  return launch_pdl(rotate_z0_kernel, grid, dim3(COPY_THREADS), 0, stream,
+                    static_cast<uint8_t*>(base), block_stride_bytes, vec_per_block,
+                    static_cast<int>(vec_per_row_head), tab);
 }
 
 cudaError_t launch_evict(void* base, int blocks, int64_t block_stride_bytes,

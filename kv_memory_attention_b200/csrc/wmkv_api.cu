@@ -12,6 +12,7 @@
 // contiguous prefix while the buffer fills.
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
@@ -32,6 +33,11 @@ struct wm_kvbuf {
   int* status = nullptr;     // device error word
   int64_t t = -1;            // current frame
   std::vector<int64_t> written;  // per block: frame of the latest write_record
+  // streaming sink (start image keys follow the window)
+  bool sink = false;
+  std::vector<double> theta;   // per dimension pair, radians per frame (0: not temporal)
+  int gap_trigger = 5, gap_target = 1;
+  int64_t z0_pos = 0;          // temporal position of the start image
 };
 
 namespace {
@@ -64,6 +70,16 @@ int raw_slot(int64_t Y, int64_t t) { return t < 1 ? -1 : static_cast<int>((t - 1
 
 int sum_slot(int64_t Y, int64_t W, int64_t f) {
   return (f < 1 || W <= Y) ? -1 : static_cast<int>((f - 1) % (W - Y));
+}
+
+void sink_table(const wm_kvbuf* h, int64_t shift, wmkv::SinkTable* tab) {
+  *tab = {};
+  for (int i = 0; i < h->d / 2; ++i) {
+    const double a = h->theta[i] * static_cast<double>(shift);
+    tab->c[i] = static_cast<float>(std::cos(a));
+    tab->s[i] = static_cast<float>(std::sin(a));
+    if (h->theta[i] != 0.0) tab->mask |= 1ull << i;
+  }
 }
 
 int64_t record_row(int64_t hw, int64_t X, int64_t Y, int64_t t) {
@@ -166,7 +182,45 @@ int wm_advance(wm_kvbuf* h, int64_t t, wm_stream_t stream) {
                                        reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e);
   }
+  if (h->sink && t >= 1) {
+    const int64_t oldest = t - h->W > 1 ? t - h->W : 1;  // oldest frame in memory
+    const int64_t gap = oldest - h->z0_pos;
+    if (gap >= h->gap_trigger) {
+      const int64_t shift = gap - h->gap_target;
+      wmkv::SinkTable tab;
+      sink_table(h, shift, &tab);
+      cudaError_t e = wmkv::launch_rotate_z0(h->buf, h->blocks, h->block_bytes, h->R, h->heads,
+                                             h->d, tab, reinterpret_cast<cudaStream_t>(stream));
+      if (e != cudaSuccess) return cuda_fail(e);
+      h->z0_pos += shift;
+    }
+  }
   h->t = t;
+  return WM_OK;
+}
+
+int wm_set_sink(wm_kvbuf* h, const float* theta, int n_pairs, int gap_trigger, int gap_target) {
+  if (!h || !theta || n_pairs != h->d / 2 || gap_target < 0 || gap_trigger <= gap_target)
+    return WM_ERR_INVALID_ARG;
+  if (h->t >= 0) return WM_ERR_STATE;
+  h->theta.assign(theta, theta + n_pairs);
+  h->gap_trigger = gap_trigger;
+  h->gap_target = gap_target;
+  h->z0_pos = 0;
+  h->sink = true;
+  return WM_OK;
+}
+
+int64_t wm_sink_position(const wm_kvbuf* h) { return h ? h->z0_pos : -1; }
+
+int wm_sink_cos_sin(const wm_kvbuf* h, int64_t shift, float* c, float* s) {
+  if (!h || !h->sink || !c || !s) return WM_ERR_INVALID_ARG;
+  wmkv::SinkTable tab;
+  sink_table(h, shift, &tab);
+  for (int i = 0; i < h->d / 2; ++i) {
+    c[i] = tab.c[i];
+    s[i] = tab.s[i];
+  }
   return WM_OK;
 }
 

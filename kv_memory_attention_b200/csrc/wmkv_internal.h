@@ -65,6 +65,17 @@ bool attend_copies_in_kernel(int d);
 cudaError_t launch_copy_pair(const void* a_src, const void* b_src, void* a_dst, void* b_dst,
                              int64_t n16, cudaStream_t stream);
 
+// Rotation of adjacent dimension pairs (at most 64 per head row).
+struct SinkTable {
+  float c[64];
+  float s[64];
+  unsigned long long mask;  // bit i: pair i turns
+};
+// Z0 key rotation in every block: rows [0, rows) of the K buffer at
+// base + b*block_stride_bytes.
+cudaError_t launch_rotate_z0(void* base, int blocks, int64_t block_stride_bytes, int64_t rows,
+                             int heads, int d, const SinkTable& tab, cudaStream_t stream);
+
 // RAW -> SUM eviction in every block of one allocation.
 //   base: the allocation; block b's K buffer at base + b*block_stride_bytes,
 //   its V buffer at + tensor_stride_bytes.  Copies `n16` chunks from

@@ -32,6 +32,10 @@ SIGNATURES = {
     "wm_write_record": (_c_int, [_vp, _c_int, _c_i64, _vp, _vp, _vp]),
     "wm_attend": (_c_int, [_vp, _c_int, _vp, _vp, _vp]),
     "wm_write_attend": (_c_int, [_vp, _c_int, _c_i64, _vp, _vp, _vp, _vp, _vp]),
+    "wm_set_sink": (_c_int, [_vp, ctypes.POINTER(ctypes.c_float), _c_int, _c_int, _c_int]),
+    "wm_sink_position": (_c_i64, [_vp]),
+    "wm_sink_cos_sin": (_c_int, [_vp, _c_i64, ctypes.POINTER(ctypes.c_float),
+                                 ctypes.POINTER(ctypes.c_float)]),
     "wm_end": (_c_i64, [_vp]),
     "wm_capacity": (_c_i64, [_vp]),
     "wm_current_frame": (_c_i64, [_vp]),
@@ -127,6 +131,22 @@ def wm_attend(h: int, block: int, Q, O, stream=None) -> None:
 def wm_write_attend(h: int, block: int, t: int, Q, K, V, O, stream=None) -> None:
     _check(LIB.wm_write_attend(h, block, t, _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _stream(stream)),
            "wm_write_attend")
+
+
+def wm_set_sink(h: int, theta, gap_trigger: int = 5, gap_target: int = 1) -> None:
+    arr = (ctypes.c_float * len(theta))(*[float(x) for x in theta])
+    _check(LIB.wm_set_sink(h, arr, len(theta), gap_trigger, gap_target), "wm_set_sink")
+
+
+def wm_sink_position(h: int) -> int:
+    return LIB.wm_sink_position(h)
+
+
+def wm_sink_cos_sin(h: int, shift: int, n_pairs: int):
+    c = (ctypes.c_float * n_pairs)()
+    s = (ctypes.c_float * n_pairs)()
+    _check(LIB.wm_sink_cos_sin(h, shift, c, s), "wm_sink_cos_sin")
+    return list(c), list(s)
 
 
 def wm_end(h: int) -> int:
@@ -232,6 +252,12 @@ class KVMemory:
 
     def end(self):
         return wm_end(self.h)
+
+    def set_sink(self, theta, gap_trigger=5, gap_target=1):
+        wm_set_sink(self.h, theta, gap_trigger, gap_target)
+
+    def sink_position(self):
+        return wm_sink_position(self.h)
 
     def sync_status(self):
         wm_sync_status(self.h)
