@@ -127,7 +127,9 @@ def test_served_single_block_steady_state(wm):
 
 DENSE_CASES = [(1, 1, 1, 64), (5, 3, 2, 64), (128, 128, 2, 64), (129, 300, 3, 64),
                (200, 129, 2, 64), (64, 1000, 1, 64), (300, 1000, 2, 128), (257, 129, 4, 128),
-               (33, 1, 2, 128), (1104, 6528, 2, 64)]
+               (33, 1, 2, 128), (1104, 6528, 2, 64),
+               # key counts around the 96-key tiles of the d = 64 kernel
+               (130, 96, 2, 64), (130, 97, 2, 64), (130, 192, 1, 64), (130, 289, 2, 64)]
 
 
 def dense_inputs(lq, lk, heads, d, tag):
