@@ -13,6 +13,11 @@ Prints ONE JSON line on rank 0.  ``value`` = frame-steps/s over all ranks
 the data path), timed with CUDA events between a barrier + synchronize on
 both sides, max over ranks.  ``--impl reference`` times the fp64 CPU oracle on
 the host cores instead (rank 0 only).
+
+At N = 1 the line also carries ``extras`` (none of them enters ``value``): the
+same frame-step replayed from CUDA graphs, the HBM throughput of the eviction
+and record-write kernels, a batch of 8 sessions, and the scaled memory (24 x
+128, W = 48) against the dense full-history attention it replaces.
 """
 from __future__ import annotations
 
@@ -244,6 +249,11 @@ def run_ours(args, world, rank, local):
     t = e2e.pop("_t")
     kv.sync_status()
 
+    # ------------------------------------------------ secondary measurements (N = 1 only)
+    extras = None
+    if world == 1 and not args.no_extras:
+        extras, t = run_extras(torch, wm, device, kv, t, Q, K, V, O, window)
+
     value = aggregate_throughput(args.steps, elapsed_ms, world)
     sustained, burst, hbm, src = peaks()
     achieved_tflops = ATTN_FLOP / (attn_avg_ms * 1e-3) / 1e12
@@ -273,6 +283,8 @@ def run_ours(args, world, rank, local):
         "gpu_launches": launches,
         "clocks": clk.summary(),
     }
+    if extras is not None:
+        line["extras"] = extras
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     if rank == 0:
@@ -347,6 +359,262 @@ def run_e2e(args, torch, wm, kv, t, rank, world, device, Qd, Kd, Vd):
             "ms_per_step": round(ms / args.steps, 4),
             "how": "pinned host Q/K/V copied in on a copy stream, O copied out on another, "
                    "overlapped with the kernels block by block", "_t": t}
+
+
+# ---------------------------------------------------------------- secondary measurements
+# Reported under "extras" at N = 1; none of them enters `value`.
+
+GRAPH_PERIOD = 66   # lcm(Y + 1, W - Y): the served slot pattern repeats every 66 frames
+
+
+def _timed(torch, fn, n):
+    """CUDA-event time of n calls of fn on the current stream, in ms per call."""
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(n):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / n
+
+
+def extra_graph(torch, kv, t, Q, K, V, O):
+    """The served frame-step replayed from CUDA graphs.
+
+    One graph per frame for GRAPH_PERIOD consecutive frames: the slots a frame
+    writes and evicts repeat with that period, so replaying the graphs in
+    order continues the rollout exactly.  Returns (result, next t).
+    """
+    cap = torch.cuda.Stream()
+    graphs = []
+    torch.cuda.synchronize()
+    for _ in range(GRAPH_PERIOD):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            s = torch.cuda.current_stream()
+            kv.advance(t, s)
+            for b in range(BLOCKS):
+                kv.write_attend(b, t, Q[b], K[b], V[b], O[b], s)
+        graphs.append(g)
+        t += 1
+
+    def cycle():
+        for g in graphs:
+            g.replay()
+
+    cycle()                                   # warm-up cycle
+    cycles = 3
+    ms = _timed(torch, cycle, cycles) / GRAPH_PERIOD
+    kv.sync_status()
+    del graphs
+    return {"value": round(1e3 / ms, 3), "unit": UNIT, "ms_per_step": round(ms, 4),
+            "steps": cycles * GRAPH_PERIOD,
+            "how": f"{GRAPH_PERIOD} frame-steps captured as one CUDA graph each "
+                   f"(29 launches), replayed in order {cycles} times after one warm-up cycle"}, t
+
+
+def extra_copies(torch, kv, t, K, V, hbm_gbs):
+    """HBM throughput of the eviction (wm_advance) and the record write
+    (wm_write_record), each launch timed alone after reading a 512 MB buffer
+    (clean lines: the L2 holds none of the copy's data and nothing dirty).
+    The rollout stays valid: every block gets its record every frame."""
+    flush = torch.empty(128 * 2 ** 20, dtype=torch.float32, device=K[0].device).fill_(1.0)
+    ev, wr = [], []
+    n = 10
+    for _ in range(n):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        flush.sum()
+        e[0].record()
+        kv.advance(t)
+        e[1].record()
+        for b in range(BLOCKS):
+            if b == 0:
+                flush.sum()
+                e[2].record()
+            kv.write_record(b, t, K[b], V[b])
+            if b == 0:
+                e[3].record()
+        ev.append(e)
+        t += 1
+    torch.cuda.synchronize()
+    kv.sync_status()
+    evict_us = statistics.median(x[0].elapsed_time(x[1]) for x in ev) * 1e3
+    write_us = statistics.median(x[2].elapsed_time(x[3]) for x in ev) * 1e3
+    del flush
+
+    def entry(kernel, nbytes, us):
+        gbs = nbytes / (us * 1e-6) / 1e9
+        return {"kernel": kernel, "bytes": nbytes, "us": round(us, 2), "GB_per_s": round(gbs, 1),
+                "frac_of_hbm": round(gbs / hbm_gbs, 3)}
+
+    return {"evict": entry("evict_kernel (28 blocks, one launch)", EVICT_BYTES, evict_us),
+            "record_write": entry("copy_pair_kernel (one block)", WRITE_BYTES, write_us),
+            "how": f"median of {n} launches, each after a 512 MB read (L2 holds no copy data); "
+                   "bytes = algorithmic read + write"}, t
+
+
+def extra_batch(torch, wm, window, device, sessions=8, steps=20):
+    """Eight independent served sessions on one stream, interleaved block by
+    block (each session: its own memory and inputs, K rows scaled per token by
+    U(0.5, 2)); aggregate frame-steps/s."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(0x5EED + 4)
+    mems, ins = [], []
+    for s in range(sessions):
+        mems.append(wm.KVMemory(BLOCKS, HEADS, D, GH, GW, X, Y, W))
+        q = [window(si.seed_for(4, s, b, 0, 0, si.T_Q)) for b in range(BLOCKS)]
+        k = [window(si.seed_for(4, s, b, 0, 0, si.T_K)) for b in range(BLOCKS)]
+        v = [window(si.seed_for(4, s, b, 0, 0, si.T_V)) for b in range(BLOCKS)]
+        for b in range(BLOCKS):
+            scale = torch.rand(R, 1, 1, generator=gen, device=device) * 1.5 + 0.5
+            k[b] = (k[b].float() * scale).to(torch.bfloat16)
+        o = [torch.empty(R, HEADS, D, dtype=torch.bfloat16, device=device) for _ in range(BLOCKS)]
+        ins.append((q, k, v, o))
+    for t in range(T_STEADY):
+        for s, m in enumerate(mems):
+            m.advance(t)
+            for b in range(BLOCKS):
+                m.write_record(b, t, ins[s][1][b], ins[s][2][b])
+    t = T_STEADY
+
+    def step():
+        nonlocal t
+        for m in mems:
+            m.advance(t)
+        for b in range(BLOCKS):
+            for s, m in enumerate(mems):
+                q, k, v, o = ins[s]
+                m.write_attend(b, t, q[b], k[b], v[b], o[b])
+        t += 1
+
+    for _ in range(3):
+        step()
+    ms = _timed(torch, step, steps)
+    for m in mems:
+        m.sync_status()
+        m.close()
+    return {"sessions": sessions, "value": round(sessions * 1e3 / ms, 3), "unit": UNIT,
+            "ms_per_step": round(ms, 4), "steps": steps,
+            "how": "8 served sessions on one stream: each frame-step advances all 8, then for "
+                   "each block runs write_attend of every session"}
+
+
+def extra_scaled(torch, wm, device, sustained, steps=3):
+    """The scaled memory (24 heads x 128, 45x80 + X=256, Y=2, W=48: 3856 queries
+    x 27,200 keys) at steady state, and the dense full-history baseline it
+    replaces (3600 queries x 180,000 keys, wm_attend_dense), 28 blocks each.
+    One set of synthetic Q/K/V serves all blocks and frames."""
+    B, H, d, gh, gw, x, y, w = 28, 24, 128, 45, 80, 256, 2, 48
+    hw = gh * gw
+    r = hw + x
+    c = r * (y + 2) + x * (w - y)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(0x5EED + 5)
+
+    def randn(*shape):
+        return torch.randn(*shape, generator=gen, device=device).to(torch.bfloat16)
+
+    kv2 = wm.KVMemory(B, H, d, gh, gw, x, y, w)
+    q, k, v = randn(r, H, d), randn(r, H, d), randn(r, H, d)
+    o = torch.empty(r, H, d, dtype=torch.bfloat16, device=device)
+    t_steady = 60
+    for t in range(t_steady):
+        kv2.advance(t)
+        for b in range(B):
+            kv2.write_record(b, t, k, v)
+    t = t_steady
+
+    # the copy kernels at this size (one eviction: 28 blocks x 256 rows of K and
+    # V; one record write: 3856 rows of K and V), each launch timed alone after
+    # a 512 MB read that leaves no copy data in L2
+    flush = torch.empty(128 * 2 ** 20, dtype=torch.float32, device=device).fill_(1.0)
+    ev = []
+    for _ in range(5):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        flush.sum()
+        e[0].record()
+        kv2.advance(t)
+        e[1].record()
+        flush.sum()
+        e[2].record()
+        kv2.write_record(0, t, k, v)
+        e[3].record()
+        for b in range(1, B):
+            kv2.write_record(b, t, k, v)
+        ev.append(e)
+        t += 1
+    torch.cuda.synchronize()
+    del flush
+    evict_us = statistics.median(e[0].elapsed_time(e[1]) for e in ev) * 1e3
+    write_us = statistics.median(e[2].elapsed_time(e[3]) for e in ev) * 1e3
+    evict_bytes = 2 * 2 * x * H * d * 2 * B
+    write_bytes = 2 * 2 * r * H * d * 2
+
+    def step():
+        nonlocal t
+        kv2.advance(t)
+        for b in range(B):
+            kv2.write_attend(b, t, q, k, v, o)
+        t += 1
+
+    step()
+    ms_s = _timed(torch, step, steps)
+    kv2.sync_status()
+    kv2.close()
+    del q, k, v, o
+
+    lk = (w + 2) * hw
+    qd, kd, vd = randn(hw, H, d), randn(lk, H, d), randn(lk, H, d)
+    od = torch.empty(hw, H, d, dtype=torch.bfloat16, device=device)
+    st = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def dense_step():
+        for _ in range(B):
+            wm.wm_attend_dense(qd, kd, vd, od, hw, lk, H, d, st)
+
+    wm.wm_attend_dense(qd, kd, vd, od, hw, lk, H, d, st)
+    ms_d = _timed(torch, dense_step, 1)
+    if int(st.item()) != 0:
+        raise RuntimeError("dense attention reported a device timeout")
+    del qd, kd, vd, od
+
+    def entry(ms, flop, n):
+        tf = flop / (ms * 1e-3) / 1e12
+        return {"ms_per_step": round(ms, 3), "frame_steps_per_s": round(1e3 / ms, 3),
+                "tflops": round(tf, 1), "frac_of_bf16_peak": round(tf / sustained, 4), "steps": n}
+
+    scaled = entry(ms_s, B * 4 * r * c * d * H, steps)
+    scaled.update({"queries": r, "keys": c, "heads": H, "head_dim": d})
+    dense = entry(ms_d, B * 4 * hw * lk * d * H, 1)
+    dense.update({"queries": hw, "keys": lk, "heads": H, "head_dim": d})
+    _, _, hbm, _ = peaks()
+    copies = {}
+    for name, kern, nbytes, us in (("evict", "evict_kernel (28 blocks, one launch)", evict_bytes, evict_us),
+                                   ("record_write", "copy_pair_kernel (one block)", write_bytes, write_us)):
+        gbs = nbytes / (us * 1e-6) / 1e9
+        copies[name] = {"kernel": kern, "bytes": nbytes, "us": round(us, 2), "GB_per_s": round(gbs, 1),
+                        "frac_of_hbm": round(gbs / hbm, 3)}
+    return {"scaled": scaled, "dense_baseline": dense, "copy_kernels_scaled": copies,
+            "speedup_vs_dense": round(ms_d / ms_s, 2),
+            "how": "frame-step = advance + 28 x write_attend (scaled) vs 28 x wm_attend_dense over "
+                   "the full history; one synthetic Q/K/V set reused by all blocks"}
+
+
+def run_extras(torch, wm, device, kv, t, Q, K, V, O, window):
+    """All secondary measurements; a section that fails reports its error."""
+    sustained, _, hbm, _ = peaks()
+    out = {}
+    for name, fn in (("graph", lambda: extra_graph(torch, kv, t, Q, K, V, O)),
+                     ("copy_kernels", lambda: extra_copies(torch, kv, t, K, V, hbm)),
+                     ("batch8", lambda: (extra_batch(torch, wm, window, device), t)),
+                     ("scaled_vs_dense", lambda: (extra_scaled(torch, wm, device, sustained), t))):
+        try:
+            out[name], t = fn()
+        except Exception as e:  # reported, not hidden: the main line stands on its own
+            out[name] = {"error": f"{type(e).__name__}: {e}"}
+            torch.cuda.synchronize()
+    return out, t
 
 
 TRAFFIC_SUMMARY = os.path.join(ROOT, "profiles", "attend_kernel_served.md")
@@ -490,6 +758,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the secondary measurements (CUDA graphs, copy kernels' HBM "
+                         "throughput, batch of 8, scaled memory vs dense baseline)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)      # at least 3 untimed warm-up steps
     world, rank, local = dist_setup()
