@@ -211,6 +211,10 @@ def test_sampled_rows_helper_is_in_range():
     (Layout(24, 42, 96, 2, 24, heads=4, d=64), range(30)),
     (Layout(3, 5, 2, 0, 4, heads=2, d=64), range(9)),
     (Layout(5, 7, 9, 2, 9, heads=2, d=128), range(14)),
+    # record and summary lengths multiples of 8: tiles run across the seams
+    # between the three key segments (short last tiles fall back)
+    (Layout(4, 4, 8, 2, 6, heads=2, d=64), range(12)),
+    (Layout(8, 10, 16, 1, 7, heads=2, d=64), range(14)),
 ])
 def test_write_attend_equals_write_then_attend(wm, L, frames):
     """One launch (keys: buffer before/after the slot + the record from the caller) gives
