@@ -163,8 +163,14 @@ WM_API int64_t wm_layout_record_row(int grid_h, int grid_w, int X, int Y, int64_
  *   O[i,h,:] = sum_j softmax_j(Q[i,h,:] . K[j,h,:] / sqrt(d)) V[j,h,:],  j < Lk,
  * Q/O device [Lq, heads, d], K/V device [Lk, heads, d], all bf16, same
  * kernel and numerics as wm_attend.  Lq >= 1, Lk >= 1, d in {64, 128}.
- * `dev_status` is an optional device int (NULL to skip) that receives
- * WM_ERR_TIMEOUT if the kernel gives up a bounded wait. */
+ * `dev_status` is an optional device int (NULL to skip) that the kernel sets
+ * to 1 if it gives up a bounded wait (about 2 s); it is not touched
+ * otherwise, so the caller zeroes it beforehand and reads it after the
+ * stream has reached the launch.
+ * Returns WM_ERR_INVALID_ARG for an empty Q or K (Lq < 1 or Lk < 1), a
+ * pointer that is not 16-byte aligned or more than 65535 heads,
+ * WM_ERR_UNSUPPORTED for another head dimension, WM_ERR_CUDA if the launch
+ * fails; nothing is launched in those cases. */
 WM_API int wm_attend_dense(const void* Q, const void* K, const void* V, void* O, int64_t Lq, int64_t Lk,
                     int heads, int d, int* dev_status, wm_stream_t stream);
 

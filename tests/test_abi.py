@@ -94,6 +94,8 @@ def test_null_handle_and_pointer_errors(wm):
     assert lib.wm_attend_dense(24, 16, 16, 16, 1, 1, 1, 64, None, None) == wm.WM_ERR_INVALID_ARG
     assert lib.wm_attend_dense(16, 16, 16, 16, 0, 1, 1, 64, None, None) == wm.WM_ERR_INVALID_ARG
     assert lib.wm_attend_dense(16, 16, 16, 16, 1, 0, 1, 64, None, None) == wm.WM_ERR_INVALID_ARG
+    assert lib.wm_attend_dense(16, 16, 16, 16, 1, 1, 65536, 64, None, None) == wm.WM_ERR_INVALID_ARG
+    assert lib.wm_attend_dense(16, 16, 16, 16, 1, 1, 1, 96, None, None) == wm.WM_ERR_UNSUPPORTED
     assert lib.wm_attend_dense(16, 16, 16, 16, 1, 1, 1, 80, None, None) == wm.WM_ERR_UNSUPPORTED
 
 
