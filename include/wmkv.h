@@ -30,8 +30,14 @@
  * caller, must be 16-byte aligned, and must stay valid until the stream
  * reaches the call; the library keeps no reference to them afterwards.
  *
- * A handle is used by one host thread at a time; the library holds no global
- * mutable state.
+ * A handle is used by one host thread at a time.  Beyond the handles, the
+ * library keeps only one-time set-up done by the first call of each kind
+ * (kernel attributes, the driver's tensor-map encoder), guarded for threads.
+ * wm_advance, wm_write_record, wm_attend and wm_write_attend make no
+ * synchronous CUDA call and allocate nothing, so once each has run once
+ * outside a capture, a sequence of them can be captured into a CUDA graph;
+ * the graph replays exactly the launches of that sequence, with its frame
+ * numbers (the slot pattern repeats every lcm(Y+1, W-Y) frames).
  */
 #ifndef WMKV_H
 #define WMKV_H
