@@ -706,21 +706,28 @@ bool encode_rows_map(CUtensorMap* m, const void* base, int64_t rows, int heads, 
   return r == CUDA_SUCCESS;
 }
 
+constexpr int MAX_DEVICES = 64;
+
 template <int D>
 cudaError_t launch_d(const AttendParams& prm, int64_t lq, int heads, cudaStream_t stream) {
   using C = Cfg<D>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(attend_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    C::SMEM_ALLOC);
+  // kernel attributes belong to a device: set them once on each device used
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES)
+    return cudaErrorInvalidDevice;
+  static std::once_flag once[MAX_DEVICES];
+  static cudaError_t attr_err[MAX_DEVICES];
+  std::call_once(once[dev], [dev] {
+    cudaError_t e = cudaFuncSetAttribute(attend_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM_ALLOC);
     // setmaxnreg.inc waits until registers are free: the launch must carry
     // exactly the budget the split assumes, or the kernel is not launched.
     cudaFuncAttributes fa;
-    if (attr_err == cudaSuccess) attr_err = cudaFuncGetAttributes(&fa, attend_kernel<D>);
-    if (attr_err == cudaSuccess && fa.numRegs != LAUNCH_REGS) attr_err = cudaErrorInvalidConfiguration;
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, attend_kernel<D>);
+    if (e == cudaSuccess && fa.numRegs != LAUNCH_REGS) e = cudaErrorInvalidConfiguration;
+    attr_err[dev] = e;
   });
-  if (attr_err != cudaSuccess) return attr_err;
+  if (attr_err[dev] != cudaSuccess) return attr_err[dev];
   dim3 grid(static_cast<unsigned>((lq + BM - 1) / BM), static_cast<unsigned>(heads));
   return launch_pdl(attend_kernel<D>, grid, dim3(NUM_THREADS), C::SMEM_ALLOC, stream, prm);
 }

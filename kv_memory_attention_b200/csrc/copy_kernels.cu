@@ -12,6 +12,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "sm100_ptx.cuh"
 #include "wmkv_internal.h"
 
@@ -111,15 +113,20 @@ __global__ void __launch_bounds__(COPY_THREADS) rotate_z0_kernel(uint8_t* base, 
   *v = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+// SM count of the current device (queried once per device, thread-safe).
 int sm_count() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
+  constexpr int MAX_DEVICES = 64;
+  static std::once_flag once[MAX_DEVICES];
+  static int count[MAX_DEVICES];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return 148;
+  std::call_once(once[dev], [dev] {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    count[dev] = n;
+  });
+  return count[dev];
 }
 
 unsigned grid_x_for(int64_t n16, int parallel_arrays) {
