@@ -30,6 +30,9 @@
  * caller, must be 16-byte aligned, and must stay valid until the stream
  * reaches the call; the library keeps no reference to them afterwards.
  *
+ * A handle belongs to the CUDA device that was current when it was created:
+ * wm_advance, wm_write_record, wm_attend and wm_write_attend return
+ * WM_ERR_STATE unless that device is current (and the stream belongs to it).
  * A handle is used by one host thread at a time.  Beyond the handles, the
  * library keeps only one-time set-up done by the first call of each kind
  * (kernel attributes, the driver's tensor-map encoder), guarded for threads.
@@ -145,7 +148,8 @@ WM_API int wm_sum_slot(const wm_kvbuf* h, int64_t f);     /* (f-1) mod (W-Y) for
  * by the handle; valid until wm_kvbuf_destroy. */
 WM_API int wm_kv_ptrs(const wm_kvbuf* h, int block, void** K, void** V);
 
-/* Synchronise the device, then read and clear the handle's device error flag:
+/* Synchronise the handle's device (the caller's current device is restored),
+ * then read and clear the handle's device error flag:
  * WM_ERR_TIMEOUT if a kernel gave up a bounded wait since the last call,
  * WM_ERR_CUDA if the synchronisation itself failed, else WM_OK. */
 WM_API int wm_sync_status(wm_kvbuf* h);

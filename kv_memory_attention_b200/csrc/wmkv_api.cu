@@ -169,9 +169,17 @@ int wm_kvbuf_destroy(wm_kvbuf* h) {
   return e == cudaSuccess ? WM_OK : cuda_fail(e);
 }
 
+// The handle's buffers live on the device that was current at creation; its
+// kernels must be launched there (another device would read memory it does
+// not own).
+static bool on_handle_device(const wm_kvbuf* h) {
+  int dev = -1;
+  return cudaGetDevice(&dev) == cudaSuccess && dev == h->device;
+}
+
 int wm_advance(wm_kvbuf* h, int64_t t, wm_stream_t stream) {
   if (!h) return WM_ERR_INVALID_ARG;
-  if (t != h->t + 1) return WM_ERR_STATE;
+  if (t != h->t + 1 || !on_handle_device(h)) return WM_ERR_STATE;
   const int64_t f = t - h->Y - 1;  // frame leaving the raw window
   if (f >= 1 && h->W > h->Y) {
     const int64_t src_row = h->R * (1 + raw_slot(h->Y, f)) + h->HW;
@@ -228,7 +236,7 @@ int wm_write_record(wm_kvbuf* h, int block, int64_t t, const void* K, const void
                     wm_stream_t stream) {
   if (!h || block < 0 || block >= h->blocks || !aligned16(K) || !aligned16(V))
     return WM_ERR_INVALID_ARG;
-  if (h->t < 0 || t != h->t) return WM_ERR_STATE;
+  if (h->t < 0 || t != h->t || !on_handle_device(h)) return WM_ERR_STATE;
   const int64_t row0 = record_row(h->HW, h->X, h->Y, t);
   uint8_t* kdst = h->buf + int64_t(block) * h->block_bytes + row0 * h->row_bytes;
   uint8_t* vdst = kdst + h->tensor_bytes;
@@ -242,7 +250,7 @@ int wm_write_record(wm_kvbuf* h, int block, int64_t t, const void* K, const void
 int wm_attend(wm_kvbuf* h, int block, const void* Q, void* O, wm_stream_t stream) {
   if (!h || block < 0 || block >= h->blocks || !aligned16(Q) || !aligned16(O))
     return WM_ERR_INVALID_ARG;
-  if (h->t < 0 || h->written[block] != h->t) return WM_ERR_STATE;
+  if (h->t < 0 || h->written[block] != h->t || !on_handle_device(h)) return WM_ERR_STATE;
   const int64_t end = end_at(h->HW, h->X, h->Y, h->W, h->t);
   const uint8_t* kbuf = h->buf + int64_t(block) * h->block_bytes;
   const uint8_t* vbuf = kbuf + h->tensor_bytes;
@@ -258,7 +266,7 @@ int wm_write_attend(wm_kvbuf* h, int block, int64_t t, const void* Q, const void
   if (!h || block < 0 || block >= h->blocks || !aligned16(Q) || !aligned16(K) || !aligned16(V) ||
       !aligned16(O))
     return WM_ERR_INVALID_ARG;
-  if (h->t < 0 || t != h->t) return WM_ERR_STATE;
+  if (h->t < 0 || t != h->t || !on_handle_device(h)) return WM_ERR_STATE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int64_t row0 = record_row(h->HW, h->X, h->Y, t);
   uint8_t* kbuf = h->buf + int64_t(block) * h->block_bytes;
@@ -306,17 +314,18 @@ int wm_kv_ptrs(const wm_kvbuf* h, int block, void** K, void** V) {
 
 int wm_sync_status(wm_kvbuf* h) {
   if (!h) return WM_ERR_INVALID_ARG;
-  cudaError_t e = cudaDeviceSynchronize();
+  // on the handle's device; the caller's current device is restored
+  int prev = 0;
+  cudaError_t e = cudaGetDevice(&prev);
+  if (e == cudaSuccess && prev != h->device) e = cudaSetDevice(h->device);
   if (e != cudaSuccess) return cuda_fail(e);
   int flag = 0;
-  e = cudaMemcpy(&flag, h->status, sizeof(int), cudaMemcpyDeviceToHost);
+  e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(&flag, h->status, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && flag != wmkv::DEV_OK) e = cudaMemset(h->status, 0, sizeof(int));
+  if (prev != h->device) cudaSetDevice(prev);
   if (e != cudaSuccess) return cuda_fail(e);
-  if (flag != wmkv::DEV_OK) {
-    e = cudaMemset(h->status, 0, sizeof(int));
-    if (e != cudaSuccess) return cuda_fail(e);
-    return WM_ERR_TIMEOUT;
-  }
-  return WM_OK;
+  return flag != wmkv::DEV_OK ? WM_ERR_TIMEOUT : WM_OK;
 }
 
 const char* wm_strerror(int code) {
