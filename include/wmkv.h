@@ -84,8 +84,8 @@ WM_API int wm_kvbuf_create(wm_kvbuf** out, int blocks, int heads, int d, int gri
 /* Free the buffers and the handle (synchronises the device first). */
 WM_API int wm_kvbuf_destroy(wm_kvbuf* h);
 
-/* Start frame t ("One buffer, no mask": when a frame falls out of the raw
- * window its summary rows are copied RAW -> SUM).  t must be 0, then 1, 2, ...
+/* Start frame t (section "One buffer, no mask": a frame that leaves the raw
+ * window keeps only its X summary rows, moved RAW -> SUM).  t must be 0, then 1, 2, ...
  * one call each, else WM_ERR_STATE.  For t >= Y+2 (and W > Y) one launch
  * copies frame t-Y-1's X summary rows of K and of V into SUM, in every block. */
 WM_API int wm_advance(wm_kvbuf* h, int64_t t, wm_stream_t stream);
@@ -118,10 +118,10 @@ WM_API int wm_write_attend(wm_kvbuf* h, int block, int64_t t, const void* Q, con
                            const void* V, void* O, wm_stream_t stream);
 
 /* Streaming sink (model card section "Running for a long time: the start
- * image follows the window"): frame ids keep growing while the start image
- * was written at id 0; whenever the gap between the start image's temporal
- * position and the oldest frame in memory (max(1, t-W) while frame t is
- * generated) reaches `gap_trigger` (the page: 5), wm_advance(t) rotates the
+ * image follows the window"): the start image's keys carry temporal
+ * position 0 while new frames get ever larger ids.  Let the gap be the
+ * distance from that position to the oldest frame kept (max(1, t-W) during
+ * frame t); when it reaches `gap_trigger` (the page: 5), wm_advance(t) rotates the
  * start image's keys (Z0 rows of K, every block) forward in place by
  * gap - gap_target frames (the page: back to a gap of 1).  Values are not
  * touched.  The page gives no rotary frequencies, so the caller passes them:

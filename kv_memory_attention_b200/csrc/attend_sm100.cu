@@ -1,8 +1,8 @@
 // Dense, unmasked softmax attention over a filled buffer prefix, for sm_100a.
 //
 // What it computes (model card "GTA world model: weights and inference code",
-// section "One buffer, no mask": one dense read of the filled prefix per
-// block, no mask): for every head h and query row i
+// section "One buffer, no mask": each block's queries attend to every row of
+// the buffer's filled prefix, unmasked): for every head h and query row i
 //     O[i,h,:] = sum_{j<lk} softmax_j(Q[i,h,:] . K[j,h,:] / sqrt(d)) V[j,h,:]
 //
 // Design (one CTA per 128-query tile and head, 384 threads = 3 warpgroups):

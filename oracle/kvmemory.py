@@ -12,10 +12,10 @@ Source: the model card "GTA world model: weights and inference code"
 What the page fixes, restated:
   * "A frame is a record": record(t) = the frame's H*W raw tokens followed by
     its X summary tokens (raw first).
-  * "What a frame attends to": while frame t is generated its tokens see
-    (1) frame t itself, (2) the last Y frames as whole records, (3) older
-    frames inside the window W as their X summary tokens only, (4) frame 0
-    (the start image) as a whole record, never evicted.
+  * "What a frame attends to": the keys visible to frame t's tokens are its
+    own record, the full records of frames t-Y..t-1, only the X summary rows
+    of the frames older than those but still inside the window W, and the
+    start image (frame 0) in full, which is never evicted.
   * "One buffer, no mask": one preallocated K/V buffer per block with regions
     | Z0: record(0) | RAW: (Y+1) rotating records | SUM: (W-Y) x X rotating
     summary rows |; reading is buffer[0:end], the filled prefix, one dense
@@ -25,8 +25,9 @@ What the page fixes, restated:
     slot and frame 28's summary takes the SUM slot of frame 6's.  Served
     numbers: 6,528 buffered keys, against 26,208 for the same span at full
     resolution.
-  * "The rest of the model", Sampling: each frame takes three denoising passes
-    plus one clean pass that rewrites the frame's entry in memory.
+  * "The rest of the model", Sampling: a frame is produced by three
+    denoising passes, after which a clean pass writes the frame's final
+    record over the same slot.
 
 Readings where the page leaves a step open (each is also listed in the design
 notes of the repository):

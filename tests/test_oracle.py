@@ -327,7 +327,7 @@ def test_stored_rotation_identity_cases_and_rounding():
 
 @pytest.mark.parametrize("layout", [SERVED, TINY, SERVED_W16])
 def test_sink_schedule_keeps_gap_between_one_and_four(layout):
-    """The gap to the oldest frame in memory reaches 5 and is brought back to 1."""
+    """Rotations fire when the gap hits the trigger (5) and leave a gap of 1."""
     z0, rotations = 0, []
     for t in range(0, 200):
         shift = sink_shift(layout, t, z0)
