@@ -681,28 +681,34 @@ def _oracle_threads():
 
 
 class OracleStepper:
-    """The fp64 oracle stepping one served block through steady-state frames.
+    """The fp64 oracle stepping one block through steady-state frames.
 
     Each ``step(budget)`` advances the oracle's memory one frame (eviction),
-    writes the block's record and runs attention for query rows (all 16
-    heads, 6,528 keys) until ``budget`` seconds of attention have been spent;
-    the time is extrapolated to a full frame-step of 28 blocks x 1104 rows.
+    writes the block's record and runs attention for query rows (all heads,
+    all keys of the filled prefix) until ``budget`` seconds of attention have
+    been spent; the time is extrapolated to a full frame-step of 28 blocks x
+    all query rows.  Default: the served shape (16 x 64, 1104 queries x 6,528
+    keys).
     """
 
-    def __init__(self):
+    def __init__(self, layout=None, config_id=CONFIG_ID, t_steady=T_STEADY):
         from oracle import FrameMemory, Layout
-        self.L = Layout(GH, GW, X, Y, W, heads=HEADS, d=D)
+        self.L = layout if layout is not None else Layout(GH, GW, X, Y, W, heads=HEADS, d=D)
+        self.config_id = config_id
         self.mem = FrameMemory(self.L, 1, track_records=False)
-        for t in range(T_STEADY):
+        L = self.L
+        for t in range(t_steady):
             self.mem.advance(t)
-            _, k, v = si.record_inputs(CONFIG_ID, 0, 0, t, 0, R, HEADS, D)
+            _, k, v = si.record_inputs(config_id, 0, 0, t, 0, L.R, L.heads, L.d)
             self.mem.write_record(0, t, k, v)
-        self.t = T_STEADY
+        self.t = t_steady
         self.next_row = 0
 
     def step(self, budget_s: float):
         from oracle import attend_memory
-        q, k, v = si.record_inputs(CONFIG_ID, 0, 0, self.t, 0, R, HEADS, D)
+        L = self.L
+        R = L.R
+        q, k, v = si.record_inputs(self.config_id, 0, 0, self.t, 0, R, L.heads, L.d)
         t0 = time.perf_counter()
         self.mem.advance(self.t)
         t_evict = time.perf_counter() - t0
@@ -726,12 +732,33 @@ class OracleStepper:
 
 def cpu_baseline(budget_s: float):
     per_step, rows, t_attn = OracleStepper().step(budget_s)
-    return {"value": round(1.0 / per_step, 6), "unit": UNIT, "cores": _oracle_threads(),
-            "kind": "oracle",
-            "sample": f"{rows} query rows x 16 heads x 6528 keys of one block ({t_attn:.1f} s fp64 numpy), "
-                      f"plus one eviction and one record write of that block's memory, "
-                      f"extrapolated to 28 blocks x 1104 rows",
-            "host_cpus": len(os.sched_getaffinity(0))}
+    out = {"value": round(1.0 / per_step, 6), "unit": UNIT, "cores": _oracle_threads(),
+           "kind": "oracle",
+           "sample": f"{rows} query rows x 16 heads x 6528 keys of one block ({t_attn:.1f} s fp64 numpy), "
+                     f"plus one eviction and one record write of that block's memory, "
+                     f"extrapolated to 28 blocks x 1104 rows",
+           "host_cpus": len(os.sched_getaffinity(0))}
+    small = max(0.5, budget_s / 4)
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            per1, rows1, t1 = OracleStepper().step(small)
+        out["one_thread"] = {"value": round(1.0 / per1, 6), "unit": UNIT, "cores": 1,
+                             "sample": f"{rows1} query rows of one served block ({t1:.1f} s), "
+                                       f"extrapolated the same way"}
+    except Exception as e:  # reported, not hidden
+        out["one_thread"] = {"error": f"{type(e).__name__}: {e}"}
+    try:
+        from oracle import Layout
+        scaled = Layout(45, 80, 256, 2, 48, heads=24, d=128)
+        per_s, rows_s, t_s = OracleStepper(scaled, config_id=5, t_steady=60).step(small)
+        out["scaled"] = {"value": round(1.0 / per_s, 6), "unit": UNIT, "cores": _oracle_threads(),
+                         "sample": f"{rows_s} query rows x 24 heads x {scaled.end(60)} keys of one "
+                                   f"scaled block ({t_s:.1f} s), plus one eviction and one record "
+                                   f"write, extrapolated to 28 blocks x {scaled.R} rows"}
+    except Exception as e:
+        out["scaled"] = {"error": f"{type(e).__name__}: {e}"}
+    return out
 
 
 def run_reference(args, world, rank):
