@@ -56,3 +56,17 @@ def test_reference_arm_under_torchrun():
     j = json.loads(lines[0])
     assert j["impl"] == "reference" and j["n_gpus"] == 2 and j["value"] > 0
     assert j["cpu_baseline"]["kind"] == "oracle" and j["e2e"]["h2d_bytes_per_step"] == 0
+    # the line carries every key of the bench contract, with our arm's metric and unit
+    sys.path.insert(0, ROOT)
+    import bench
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config"):
+        assert key in j, key
+    assert j["metric"] == bench.METRIC and j["unit"] == bench.UNIT
+    assert j["higher_is_better"] is True and j["steps"] == 1 and j["warmup"] == 3
+    assert j["config"]["workload"] == bench.WORKLOAD
+    for key in ("value", "unit", "cores", "kind", "sample"):
+        assert key in j["cpu_baseline"], key
+    assert j["cpu_baseline"]["value"] == j["value"] and j["cpu_baseline"]["cores"] >= 1
+    assert j["e2e"] == {"value": j["value"], "unit": j["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
