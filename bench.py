@@ -730,6 +730,18 @@ class OracleStepper:
         return per_step, rows_done, t_attn
 
 
+def _cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.lower().startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def cpu_baseline(budget_s: float):
     per_step, rows, t_attn = OracleStepper().step(budget_s)
     out = {"value": round(1.0 / per_step, 6), "unit": UNIT, "cores": _oracle_threads(),
@@ -737,7 +749,7 @@ def cpu_baseline(budget_s: float):
            "sample": f"{rows} query rows x 16 heads x 6528 keys of one block ({t_attn:.1f} s fp64 numpy), "
                      f"plus one eviction and one record write of that block's memory, "
                      f"extrapolated to 28 blocks x 1104 rows",
-           "host_cpus": len(os.sched_getaffinity(0))}
+           "host_cpus": len(os.sched_getaffinity(0)), "cpu_model": _cpu_model()}
     small = max(0.5, budget_s / 4)
     try:
         from threadpoolctl import threadpool_limits
