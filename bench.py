@@ -800,6 +800,7 @@ def run_reference(args, world, rank):
                        "grid": f"{GH}x{GW}", "X": X, "Y": Y, "W": W, "queries": R, "keys": C,
                        "parallelism": "host cores (fp64 oracle)"},
             "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "cpu_model": _cpu_model(),
                              "sample": f"per step about {budget:.2f} s of query rows of one block "
                                        f"({rows_total} rows in all) plus one eviction and one record "
                                        f"write, extrapolated to a full 28-block frame-step"},
