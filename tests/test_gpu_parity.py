@@ -8,7 +8,7 @@ import pytest
 
 import seeded_inputs as si
 from oracle import FrameMemory, Layout, SERVED, TINY, attend, attend_bits, attend_memory
-from gpu_util import (assert_attn_close, attn_errors, dev, host_bits, require_gpu, sample_rows,
+from gpu_util import (assert_attn_close, dev, host_bits, require_gpu, sample_rows,
                       torch)
 
 pytestmark = pytest.mark.gpu

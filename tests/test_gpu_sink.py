@@ -5,7 +5,7 @@ import numpy as np
 import pytest
 
 import seeded_inputs as si
-from oracle import FrameMemory, Layout, SERVED, attend_memory, rotation_cos_sin, sink_shift
+from oracle import FrameMemory, Layout, attend_memory, rotation_cos_sin
 from gpu_util import assert_attn_close, dev, host_bits, require_gpu, sample_rows, torch
 
 pytestmark = pytest.mark.gpu

@@ -18,7 +18,7 @@ import numpy as np
 import pytest
 
 import seeded_inputs as si
-from oracle import FrameMemory, Layout, SCALED, SERVED, attend, attend_memory
+from oracle import FrameMemory, SCALED, SERVED, attend, attend_memory
 from gpu_util import DevicePool, assert_attn_close, host_bits, require_gpu, sample_rows, torch
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
