@@ -13,6 +13,9 @@ import importlib
 def __getattr__(name):
     if name.startswith("__"):
         raise AttributeError(name)
+    if name == "build":
+        # the build step must import without the library it builds
+        return importlib.import_module(".build", __name__)
     mod = importlib.import_module(".wmkv", __name__)
     try:
         return getattr(mod, name)
