@@ -14,17 +14,32 @@ the data path), timed with CUDA events between a barrier + synchronize on
 both sides, max over ranks.  ``--impl reference`` times the fp64 CPU oracle on
 the host cores instead (rank 0 only).
 
-At N = 1 the line also carries ``extras`` (none of them enters ``value``): the
-median of 5 separate runs of the same frame-step, the frame-step replayed
-from CUDA graphs, the HBM throughput of the eviction
-and record-write kernels, a batch of 8 sessions, and the scaled memory (24 x
-128, W = 48) against the dense full-history attention it replaces.
+One frame-step is one pass per frame (one record write and one attention
+per block); the served pattern of four passes per frame (three denoising
+passes and the clean rewrite) is timed as well, under ``extras``.
+
+At N = 1 the line also carries ``long_run`` (median of 5 separate runs of 200
+frame-steps) and ``extras`` (none of them enters ``value``): the frame-step
+replayed from CUDA graphs, the four-pass served frame, the HBM throughput of
+the eviction and record-write kernels, a batch of 8 sessions, and the scaled
+memory (24 x 128, W = 48) against the dense full-history attention it
+replaces.  On rank 0 at N = 1 the CPU-baseline leg times the fp64 oracle on
+one block and, before the timed region, compares the GPU path with it on the
+same inputs (every byte of the block's buffers, sampled attention rows); a
+mismatch stops the run.
+
+``--ncu-csv FILE --ncu-out FILE`` only summarises an ncu CSV capture (per
+kernel: launches, total time, share, per-launch metrics, and the digest of
+the attention kernel's sources) into JSON for ``profiles/``; it needs no GPU.
 """
 from __future__ import annotations
 
 import argparse
+import csv
+import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -54,15 +69,141 @@ WORKLOAD = (f"served frame-step: advance (evict) + {BLOCKS} x write_attend (reco
             f"grid {GH}x{GW} + X={X}, Y={Y}, W={W}, {HEADS} heads x {D}, "
             f"{R} queries x {C} keys, steady state t>={T_STEADY}, one session per GPU")
 CONFIG_ID = 3
+# a timed region at least this long runs at the power-capped (sustained) clock
+SUSTAINED_REGION_S = 2.0
+
+PROFILES = os.path.join(ROOT, "profiles")
+TRAFFIC_JSON = os.path.join(PROFILES, "attend_kernel_served.json")
+LAUNCHES_JSON = os.path.join(PROFILES, "frame_step_launches_served.json")
+CSRC = os.path.join(ROOT, "kv_memory_attention_b200", "csrc")
+# the files the attention kernel is compiled from
+ATTEND_SOURCES = ("attend_sm100.cu", "sm100_ptx.cuh", "wmkv_internal.h")
 
 
-def peaks():
+def config_dict(world: int) -> dict:
+    """The workload, identical for both arms."""
+    return {"workload": WORKLOAD, "blocks": BLOCKS, "heads": HEADS, "head_dim": D,
+            "grid": f"{GH}x{GW}", "X": X, "Y": Y, "W": W, "queries": R, "keys": C,
+            "passes_per_frame": 1,
+            "parallelism": f"replicas x{world} (independent sessions)",
+            "l2": "no flush: per step the 28 blocks touch 748 MB of K/V buffers + 190 MB of "
+                  "inputs, far above the 126 MB L2"}
+
+
+def peaks() -> dict:
+    """Roofline denominators: the driver's measured peaks, else the recipe's fallback."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             p = json.load(f)
-        return p["bf16_tflops_sustained"], p["bf16_tflops"], p["hbm_gbs"], "measured"
+        return {"sustained": float(p["bf16_tflops_sustained"]), "burst": float(p["bf16_tflops"]),
+                "hbm": float(p["hbm_gbs"]), "source": "measured"}
     except Exception:
-        return 1400.0, 1590.0, 6650.0, "fallback"
+        return {"sustained": 1400.0, "burst": 1590.0, "hbm": 6650.0, "source": "fallback"}
+
+
+def source_digest() -> str:
+    """sha256 prefix of the attention kernel's source files (in a fixed order)."""
+    h = hashlib.sha256()
+    for name in ATTEND_SOURCES:
+        with open(os.path.join(CSRC, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+# ---------------------------------------------------------------- ncu summaries
+
+_TIME_UNITS = {"nsecond": 1e-3, "usecond": 1.0, "msecond": 1e3, "second": 1e6}
+_BYTE_UNITS = {"byte": 1.0, "kbyte": 1e3, "mbyte": 1e6, "gbyte": 1e9,
+               "kibyte": 1024.0, "mibyte": 1024.0 ** 2, "gibyte": 1024.0 ** 3}
+
+
+def _kernel_short_name(name: str) -> str:
+    """'void ns::(anonymous namespace)::attend_kernel<64>(ns::P)' -> 'attend_kernel<64>'."""
+    m = re.search(r"([A-Za-z_]\w*(?:<[^()]*>)?)\s*\(", name)
+    return m.group(1) if m else name.strip()
+
+
+def summarize_ncu_csv(path: str, command: str) -> dict:
+    """Per-kernel summary of an ncu ``--csv`` capture (one row per launch and metric).
+
+    Times are converted to microseconds and byte counts to bytes; every other
+    metric is averaged per launch as printed."""
+    with open(path, newline="") as f:
+        lines = [ln for ln in f if not ln.startswith("==")]
+    rows = list(csv.reader(lines))
+    head = next(i for i, r in enumerate(rows) if "Kernel Name" in r and "Metric Name" in r)
+    cols = {name: i for i, name in enumerate(rows[head])}
+    launches = {}
+    for r in rows[head + 1:]:
+        if len(r) < len(cols):
+            continue
+        lid = r[cols["ID"]]
+        kname = _kernel_short_name(r[cols["Kernel Name"]])
+        metric = r[cols["Metric Name"]]
+        unit = r[cols["Metric Unit"]].strip().lower()
+        try:
+            val = float(r[cols["Metric Value"]].replace(",", ""))
+        except ValueError:
+            continue
+        if unit in _TIME_UNITS:
+            val *= _TIME_UNITS[unit]
+        elif unit in _BYTE_UNITS:
+            val *= _BYTE_UNITS[unit]
+        launches.setdefault(lid, {"kernel": kname, "metrics": {}})["metrics"][metric] = val
+    per = {}
+    for rec in launches.values():
+        k = per.setdefault(rec["kernel"], {"launches": 0, "sums": {}})
+        k["launches"] += 1
+        for m, v in rec["metrics"].items():
+            k["sums"][m] = k["sums"].get(m, 0.0) + v
+    total_us = sum(k["sums"].get("gpu__time_duration.sum", 0.0) for k in per.values())
+    kernels = []
+    for name, k in sorted(per.items(), key=lambda kv: -kv[1]["sums"].get("gpu__time_duration.sum", 0)):
+        n = k["launches"]
+        entry = {"kernel": name, "launches": n}
+        t = k["sums"].get("gpu__time_duration.sum")
+        if t is not None:
+            entry.update({"total_us": round(t, 3), "avg_us": round(t / n, 3),
+                          "share": round(t / total_us, 4) if total_us else None})
+        for m, v in sorted(k["sums"].items()):
+            if m != "gpu__time_duration.sum":
+                entry[m + " (per launch)"] = v / n
+        rd = k["sums"].get("dram__bytes_read.sum")
+        wr = k["sums"].get("dram__bytes_write.sum")
+        if rd is not None and wr is not None:
+            entry["dram_bytes_per_launch"] = int(round((rd + wr) / n))
+        kernels.append(entry)
+    return {"command": command, "source_sha256": source_digest(),
+            "captured_launches": len(launches), "kernels": kernels,
+            "note": "ncu replays each launch cold and serialised: compare shares, not absolute times"}
+
+
+def _profile_entry(path: str, prefix: str):
+    """The kernel entry whose name starts with ``prefix`` in a summary JSON that
+    was taken from the current attention sources, else None."""
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        if j.get("source_sha256") != source_digest():
+            return None
+        for k in j["kernels"]:
+            if k["kernel"].startswith(prefix):
+                return k
+    except Exception:
+        return None
+    return None
+
+
+def load_traffic():
+    """DRAM bytes (read + write) per attention launch from the committed ncu JSON,
+    or None when the kernel sources changed since it was captured."""
+    k = _profile_entry(TRAFFIC_JSON, "attend_kernel<64>")
+    return None if k is None else k.get("dram_bytes_per_launch")
+
+
+def load_ncu_share():
+    k = _profile_entry(LAUNCHES_JSON, "attend_kernel<64>")
+    return None if k is None else k.get("share")
 
 
 # ---------------------------------------------------------------- clocks
@@ -160,6 +301,19 @@ def barrier(world):
         dist.barrier()
 
 
+def attention_launch_time(step_ms_total: float, evict_ms_total: float, steps: int) -> float:
+    """Average attention launch duration (ms) inside a run of frame-steps: the run's
+    time minus its evictions, over its 28 launches per step."""
+    return (step_ms_total - evict_ms_total) / (BLOCKS * steps)
+
+
+def choose_peak(pk: dict, region_s: float):
+    """The burst peak for a region shorter than SUSTAINED_REGION_S, else the sustained one."""
+    if region_s >= SUSTAINED_REGION_S:
+        return pk["sustained"], "bf16_tflops_sustained"
+    return pk["burst"], "bf16_tflops"
+
+
 # ---------------------------------------------------------------- our arm
 
 def run_ours(args, world, rank, local):
@@ -168,6 +322,12 @@ def run_ours(args, world, rank, local):
     device = torch.device("cuda", local)
     init_pg(world, "nccl")
     import kv_memory_attention_b200 as wm
+
+    # CPU baseline (rank 0, N = 1): the oracle timed on host cores, and the GPU
+    # path checked against it on the same inputs before anything is timed
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_and_parity(args.cpu_seconds, torch, wm)
 
     kv = wm.KVMemory(BLOCKS, HEADS, D, GH, GW, X, Y, W)
     pool = torch.from_numpy(si._pool()["bf16"].view(np.int16)).to(device).view(torch.bfloat16)
@@ -197,13 +357,13 @@ def run_ours(args, world, rank, local):
 
     def step(t, ev=None):
         # one launch per block: the record write and the attention are fused
+        if ev is not None:
+            ev[0].record(stream)
         kv.advance(t, stream)
+        if ev is not None:
+            ev[1].record(stream)
         for b in range(BLOCKS):
-            if ev is not None:
-                ev[b][0].record(stream)
             kv.write_attend(b, t, Q[b], K[b], V[b], O[b], stream)
-            if ev is not None:
-                ev[b][1].record(stream)
 
     for _ in range(args.warmup):
         step(t)
@@ -230,64 +390,73 @@ def run_ours(args, world, rank, local):
     elapsed_ms = max_over_ranks(start.elapsed_time(stop), world, device)
     launches = args.steps * (1 + BLOCKS)
 
-    # ------------------------------------------------ per-launch attention time (roofline)
-    # A second timed pass of the same steps with an event pair around every
-    # attend launch, on the launching stream.
+    # ------------------------------------------------ attention launch time (roofline)
+    # The same steps again with an event pair around each eviction only: the
+    # attention launches keep overlapping each other, and their average
+    # duration is the run's time minus the evictions, over 28 per step.
     n_rf = max(1, min(args.steps, 200))
-    ev_attn = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in range(BLOCKS)] for _ in range(n_rf)]
+    ev_evict = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(n_rf)]
+    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
+    r0.record(stream)
     for s in range(n_rf):
-        step(t, ev_attn[s])
+        step(t, ev_evict[s])
         t += 1
+    r1.record(stream)
     torch.cuda.synchronize()
     kv.sync_status()
-    attn_ms = [a.elapsed_time(b) for row in ev_attn for (a, b) in row]
-    attn_avg_ms = max_over_ranks(statistics.mean(attn_ms), world, device)
+    rf_total_ms = r0.elapsed_time(r1)
+    evict_ms = sum(a.elapsed_time(b) for a, b in ev_evict)
+    attn_avg_ms = max_over_ranks(attention_launch_time(rf_total_ms, evict_ms, n_rf), world, device)
 
     # ------------------------------------------------ end to end: host buffers through the ABI
     e2e = run_e2e(args, torch, wm, kv, t, rank, world, device, Q, K, V)
     t = e2e.pop("_t")
     kv.sync_status()
 
-    # ------------------------------------------------ secondary measurements (N = 1 only)
-    extras = None
+    # ------------------------------------------------ longer runs and secondary measurements (N = 1)
+    long_run, extras = None, None
     if world == 1 and not args.no_extras:
+        long_run, t = extra_runs(torch, kv, t, Q, K, V, O)
         extras, t = run_extras(torch, wm, device, kv, t, Q, K, V, O, window)
 
     value = aggregate_throughput(args.steps, elapsed_ms, world)
-    sustained, burst, hbm, src = peaks()
+    pk = peaks()
+    peak, peak_name = choose_peak(pk, rf_total_ms / 1e3)
     achieved_tflops = ATTN_FLOP / (attn_avg_ms * 1e-3) / 1e12
     step_tflops = BLOCKS * ATTN_FLOP * args.steps / (elapsed_ms / 1e3) / 1e12
-    traffic = load_traffic()
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(elapsed_ms / args.steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "blocks": BLOCKS, "heads": HEADS, "head_dim": D,
-                   "grid": f"{GH}x{GW}", "X": X, "Y": Y, "W": W, "queries": R, "keys": C,
-                   "parallelism": f"replicas x{world} (independent sessions)",
-                   "l2": "no flush: per step the 28 blocks touch 748 MB of K/V buffers + 190 MB of "
-                         "inputs, far above the 126 MB L2"},
+        "config": config_dict(world),
         "tflops_per_step": round(step_tflops, 1),
-        "frac_of_bf16_peak_step": round(step_tflops / sustained, 4),
-        "served_frames_per_s": round(value / 4, 3),
+        "frac_of_bf16_peak_step": round(step_tflops / peak, 4),
         "roofline": {"kernel": "attend_kernel<64> (fused record write)", "bound": "tensor",
-                     "achieved": round(achieved_tflops, 1), "peak": sustained, "unit": "TFLOP/s",
-                     "frac": round(achieved_tflops / sustained, 4),
-                     "peak_source": f"bf16_tflops_sustained ({src})",
+                     "achieved": round(achieved_tflops, 1), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved_tflops / peak, 4),
+                     "peak_source": f"{peak_name} ({pk['source']}); timed region "
+                                    f"{rf_total_ms:.1f} ms",
+                     "frac_of_sustained": round(achieved_tflops / pk["sustained"], 4),
                      "avg_launch_us": round(attn_avg_ms * 1e3, 2),
-                     "launches_timed": n_rf * BLOCKS,
-                     "flop_per_launch": ATTN_FLOP, "traffic": traffic},
+                     "how": f"{n_rf} frame-steps with events around each eviction only: "
+                            f"(run time - evictions) / ({BLOCKS} x {n_rf}) launches",
+                     "run_ms": round(rf_total_ms, 3), "evict_ms": round(evict_ms, 3),
+                     "share_from_events": round(1.0 - evict_ms / rf_total_ms, 4),
+                     "ncu_share": load_ncu_share(),
+                     "flop_per_launch": ATTN_FLOP, "traffic": load_traffic()},
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clk.summary(),
     }
+    if long_run is not None:
+        line["long_run"] = long_run
     if extras is not None:
         line["extras"] = extras
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
     if rank == 0:
         print(json.dumps(line), flush=True)
     kv.close()
@@ -355,15 +524,32 @@ def run_e2e(args, torch, wm, kv, t, rank, world, device, Qd, Kd, Vd):
     barrier(world)
     ms = max_over_ranks(start.elapsed_time(stop), world, device)
     nbytes = R * HEADS * D * 2
+    h2d = 3 * BLOCKS * nbytes
+    # the host link alone: the same bytes in one pinned host -> device copy
+    big_h = torch.empty(h2d, dtype=torch.uint8).pin_memory()
+    big_d = torch.empty(h2d, dtype=torch.uint8, device=device)
+    big_d.copy_(big_h, non_blocking=True)
+    l0, l1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    l0.record()
+    for _ in range(5):
+        big_d.copy_(big_h, non_blocking=True)
+    l1.record()
+    torch.cuda.synchronize()
+    link_gbs = 5 * h2d / (l0.elapsed_time(l1) * 1e-3) / 1e9
+    del big_h, big_d
     return {"value": round(world * args.steps / (ms / 1e3), 3), "unit": UNIT,
-            "h2d_bytes_per_step": 3 * BLOCKS * nbytes, "d2h_bytes_per_step": BLOCKS * nbytes,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": BLOCKS * nbytes,
             "ms_per_step": round(ms / args.steps, 4),
+            "h2d_link_GB_per_s": round(link_gbs, 1),
+            "h2d_bound_ms_per_step": round(h2d / (link_gbs * 1e9) * 1e3, 4),
             "how": "pinned host Q/K/V (one buffer per block) copied in on a copy stream, O copied "
-                   "out on another, overlapped with the kernels block by block", "_t": t}
+                   "out on another, overlapped with the kernels block by block; the link figure is "
+                   "one pinned copy of the same bytes", "_t": t}
 
 
 # ---------------------------------------------------------------- secondary measurements
-# Reported under "extras" at N = 1; none of them enters `value`.
+# Reported under "long_run" / "extras" at N = 1; none of them enters `value`.
 
 GRAPH_PERIOD = 66   # lcm(Y + 1, W - Y): the served slot pattern repeats every 66 frames
 
@@ -429,7 +615,26 @@ def extra_runs(torch, kv, t, Q, K, V, O, runs=5, steps=200):
         vals.append(1e3 / _timed(torch, one, steps))
     kv.sync_status()
     return {"runs": runs, "steps_each": steps, "median": round(statistics.median(vals), 3),
-            "min": round(min(vals), 3), "max": round(max(vals), 3), "unit": UNIT}, t
+            "min": round(min(vals), 3), "max": round(max(vals), 3), "unit": UNIT,
+            "tflops_per_step_median": round(BLOCKS * ATTN_FLOP * statistics.median(vals) / 1e12, 1)}, t
+
+
+def extra_four_pass(torch, kv, t, Q, K, V, O, frames=50):
+    """The served frame as the model runs it: one advance, then four passes
+    (three denoising passes and the clean rewrite), each writing every block's
+    record into the same slot and attending; frames per second measured."""
+    def frame():
+        nonlocal t
+        kv.advance(t)
+        for _ in range(4):
+            for b in range(BLOCKS):
+                kv.write_attend(b, t, Q[b], K[b], V[b], O[b])
+        t += 1
+    frame()
+    ms = _timed(torch, frame, frames)
+    kv.sync_status()
+    return {"value": round(1e3 / ms, 3), "unit": "frames/s (4 passes each)", "ms_per_frame": round(ms, 4),
+            "frames": frames, "launches_per_frame": 1 + 4 * BLOCKS}, t
 
 
 def extra_copies(torch, kv, t, K, V, hbm_gbs):
@@ -469,7 +674,7 @@ def extra_copies(torch, kv, t, K, V, hbm_gbs):
     return {"evict": entry("evict_kernel (28 blocks, one launch)", EVICT_BYTES, evict_us),
             "record_write": entry("copy_pair_kernel (one block)", WRITE_BYTES, write_us),
             "how": f"median of {n} launches, each after a 512 MB read (L2 holds no copy data); "
-                   "bytes = algorithmic read + write"}, t
+                   "bytes = algorithmic read + write; CUDA events around one launch"}, t
 
 
 def extra_batch(torch, wm, window, device, sessions=8, steps=20):
@@ -518,11 +723,12 @@ def extra_batch(torch, wm, window, device, sessions=8, steps=20):
                    "each block runs write_attend of every session"}
 
 
-def extra_scaled(torch, wm, device, sustained, steps=3):
+def extra_scaled(torch, wm, device, pk, steps=3):
     """The scaled memory (24 heads x 128, 45x80 + X=256, Y=2, W=48: 3856 queries
     x 27,200 keys) at steady state, and the dense full-history baseline it
     replaces (3600 queries x 180,000 keys, wm_attend_dense), 28 blocks each.
-    One set of synthetic Q/K/V serves all blocks and frames."""
+    Every block has its own inputs: windows at different offsets of one random
+    pool per tensor (4,096 rows apart for the dense keys and values)."""
     B, H, d, gh, gw, x, y, w = 28, 24, 128, 45, 80, 256, 2, 48
     hw = gh * gw
     r = hw + x
@@ -533,14 +739,18 @@ def extra_scaled(torch, wm, device, sustained, steps=3):
     def randn(*shape):
         return torch.randn(*shape, generator=gen, device=device).to(torch.bfloat16)
 
+    def windows(pool, rows, step):
+        return [pool[b * step:b * step + rows] for b in range(B)]
+
     kv2 = wm.KVMemory(B, H, d, gh, gw, x, y, w)
-    q, k, v = randn(r, H, d), randn(r, H, d), randn(r, H, d)
+    qp, kp, vp = (randn(r + (B - 1) * 64, H, d) for _ in range(3))
+    q, k, v = windows(qp, r, 64), windows(kp, r, 64), windows(vp, r, 64)
     o = torch.empty(r, H, d, dtype=torch.bfloat16, device=device)
     t_steady = 60
     for t in range(t_steady):
         kv2.advance(t)
         for b in range(B):
-            kv2.write_record(b, t, k, v)
+            kv2.write_record(b, t, k[b], v[b])
     t = t_steady
 
     # the copy kernels at this size (one eviction: 28 blocks x 256 rows of K and
@@ -556,10 +766,10 @@ def extra_scaled(torch, wm, device, sustained, steps=3):
         e[1].record()
         flush.sum()
         e[2].record()
-        kv2.write_record(0, t, k, v)
+        kv2.write_record(0, t, k[0], v[0])
         e[3].record()
         for b in range(1, B):
-            kv2.write_record(b, t, k, v)
+            kv2.write_record(b, t, k[b], v[b])
         ev.append(e)
         t += 1
     torch.cuda.synchronize()
@@ -573,98 +783,70 @@ def extra_scaled(torch, wm, device, sustained, steps=3):
         nonlocal t
         kv2.advance(t)
         for b in range(B):
-            kv2.write_attend(b, t, q, k, v, o)
+            kv2.write_attend(b, t, q[b], k[b], v[b], o)
         t += 1
 
     step()
     ms_s = _timed(torch, step, steps)
     kv2.sync_status()
     kv2.close()
-    del q, k, v, o
+    del q, k, v, o, qp, kp, vp
 
     lk = (w + 2) * hw
-    qd, kd, vd = randn(hw, H, d), randn(lk, H, d), randn(lk, H, d)
+    qdp, kdp, vdp = randn(hw + (B - 1) * 64, H, d), randn(lk + (B - 1) * 4096, H, d), \
+        randn(lk + (B - 1) * 4096, H, d)
+    qd, kd, vd = windows(qdp, hw, 64), windows(kdp, lk, 4096), windows(vdp, lk, 4096)
     od = torch.empty(hw, H, d, dtype=torch.bfloat16, device=device)
     st = torch.zeros(1, dtype=torch.int32, device=device)
 
     def dense_step():
-        for _ in range(B):
-            wm.wm_attend_dense(qd, kd, vd, od, hw, lk, H, d, st)
+        for b in range(B):
+            wm.wm_attend_dense(qd[b], kd[b], vd[b], od, hw, lk, H, d, st)
 
-    wm.wm_attend_dense(qd, kd, vd, od, hw, lk, H, d, st)
+    wm.wm_attend_dense(qd[0], kd[0], vd[0], od, hw, lk, H, d, st)
     ms_d = _timed(torch, dense_step, 1)
     if int(st.item()) != 0:
         raise RuntimeError("dense attention reported a device timeout")
-    del qd, kd, vd, od
+    del qd, kd, vd, od, qdp, kdp, vdp
 
     def entry(ms, flop, n):
         tf = flop / (ms * 1e-3) / 1e12
+        peak, name = choose_peak(pk, ms * n / 1e3)
         return {"ms_per_step": round(ms, 3), "frame_steps_per_s": round(1e3 / ms, 3),
-                "tflops": round(tf, 1), "frac_of_bf16_peak": round(tf / sustained, 4), "steps": n}
+                "tflops": round(tf, 1), "frac_of_bf16_peak": round(tf / peak, 4),
+                "peak": f"{name} ({pk['source']})", "steps": n}
 
     scaled = entry(ms_s, B * 4 * r * c * d * H, steps)
     scaled.update({"queries": r, "keys": c, "heads": H, "head_dim": d})
     dense = entry(ms_d, B * 4 * hw * lk * d * H, 1)
     dense.update({"queries": hw, "keys": lk, "heads": H, "head_dim": d})
-    _, _, hbm, _ = peaks()
     copies = {}
     for name, kern, nbytes, us in (("evict", "evict_kernel (28 blocks, one launch)", evict_bytes, evict_us),
                                    ("record_write", "copy_pair_kernel (one block)", write_bytes, write_us)):
         gbs = nbytes / (us * 1e-6) / 1e9
         copies[name] = {"kernel": kern, "bytes": nbytes, "us": round(us, 2), "GB_per_s": round(gbs, 1),
-                        "frac_of_hbm": round(gbs / hbm, 3)}
+                        "frac_of_hbm": round(gbs / pk["hbm"], 3)}
     return {"scaled": scaled, "dense_baseline": dense, "copy_kernels_scaled": copies,
             "speedup_vs_dense": round(ms_d / ms_s, 2),
             "how": "frame-step = advance + 28 x write_attend (scaled) vs 28 x wm_attend_dense over "
-                   "the full history; one synthetic Q/K/V set reused by all blocks"}
+                   "the full history; per-block inputs are windows of one random pool per tensor"}
 
 
 def run_extras(torch, wm, device, kv, t, Q, K, V, O, window):
     """All secondary measurements; a section that fails reports its error."""
-    sustained, _, hbm, _ = peaks()
+    pk = peaks()
     out = {}
-    for name, fn in (("median_of_5_runs", lambda: extra_runs(torch, kv, t, Q, K, V, O)),
-                     ("graph", lambda: extra_graph(torch, kv, t, Q, K, V, O)),
-                     ("copy_kernels", lambda: extra_copies(torch, kv, t, K, V, hbm)),
+    for name, fn in (("graph", lambda: extra_graph(torch, kv, t, Q, K, V, O)),
+                     ("four_pass_frame", lambda: extra_four_pass(torch, kv, t, Q, K, V, O)),
+                     ("copy_kernels", lambda: extra_copies(torch, kv, t, K, V, pk["hbm"])),
                      ("batch8", lambda: (extra_batch(torch, wm, window, device), t)),
-                     ("scaled_vs_dense", lambda: (extra_scaled(torch, wm, device, sustained), t))):
+                     ("scaled_vs_dense", lambda: (extra_scaled(torch, wm, device, pk), t))):
         try:
             out[name], t = fn()
         except Exception as e:  # reported, not hidden: the main line stands on its own
             out[name] = {"error": f"{type(e).__name__}: {e}"}
             torch.cuda.synchronize()
     return out, t
-
-
-TRAFFIC_SUMMARY = os.path.join(ROOT, "profiles", "attend_kernel_served.md")
-ATTEND_SOURCE = os.path.join(ROOT, "kv_memory_attention_b200", "csrc", "attend_sm100.cu")
-
-
-def source_digest() -> str:
-    import hashlib
-    with open(ATTEND_SOURCE, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
-
-
-def load_traffic():
-    """DRAM bytes per attend launch from the committed ncu summary.
-
-    The summary records the sha256 prefix of the kernel source it was taken
-    from (``source_sha256: ...``) and ``dram_bytes_per_launch: N``; if the
-    source has changed since, the figure is stale and null is reported.
-    """
-    try:
-        fields = {}
-        with open(TRAFFIC_SUMMARY) as f:
-            for ln in f:
-                if ":" in ln:
-                    k, v = ln.split(":", 1)
-                    fields[k.strip().strip("-* `")] = v.strip().strip("`")
-        if fields.get("source_sha256") != source_digest():
-            return None
-        return int(float(fields["dram_bytes_per_launch"]))
-    except Exception:
-        return None
 
 
 # ---------------------------------------------------------------- CPU oracle
@@ -704,11 +886,15 @@ class OracleStepper:
         self.t = t_steady
         self.next_row = 0
 
+    def inputs(self, t):
+        L = self.L
+        return si.record_inputs(self.config_id, 0, 0, t, 0, L.R, L.heads, L.d)
+
     def step(self, budget_s: float):
         from oracle import attend_memory
         L = self.L
-        R = L.R
-        q, k, v = si.record_inputs(self.config_id, 0, 0, self.t, 0, R, L.heads, L.d)
+        R_ = L.R
+        q, k, v = self.inputs(self.t)
         t0 = time.perf_counter()
         self.mem.advance(self.t)
         t_evict = time.perf_counter() - t0
@@ -717,8 +903,8 @@ class OracleStepper:
         t_write = time.perf_counter() - t0
         rows_done, t_attn = 0, 0.0
         while True:
-            rows = (np.arange(self.next_row, self.next_row + 128)) % R
-            self.next_row = (self.next_row + 128) % R
+            rows = (np.arange(self.next_row, self.next_row + 128)) % R_
+            self.next_row = (self.next_row + 128) % R_
             t0 = time.perf_counter()
             attend_memory(self.mem, 0, q, rows=rows)
             t_attn += time.perf_counter() - t0
@@ -726,8 +912,9 @@ class OracleStepper:
             if t_attn >= budget_s:
                 break
         self.t += 1
-        per_step = BLOCKS * (R * t_attn / rows_done + t_write) + t_evict
-        return per_step, rows_done, t_attn
+        per_step = BLOCKS * (R_ * t_attn / rows_done + t_write) + t_evict
+        spent = t_evict + t_write + t_attn
+        return per_step, rows_done, t_attn, spent
 
 
 def _cpu_model() -> str:
@@ -742,19 +929,77 @@ def _cpu_model() -> str:
     return platform.processor() or "unknown"
 
 
-def cpu_baseline(budget_s: float):
-    per_step, rows, t_attn = OracleStepper().step(budget_s)
+def gpu_parity_on_stepper(stepper, torch, wm):
+    """The GPU path (wm_write_attend, the call the bench times) on the inputs
+    the oracle stepper is about to use for its next frame, compared with the
+    oracle: every byte of the block's K/V buffers, and sampled attention rows
+    (all heads) within max-abs 2e-2 and relative L2 5e-3.  Raises on a mismatch."""
+    from oracle import attend_memory
+    L = stepper.L
+    kv = wm.KVMemory(1, L.heads, L.d, L.grid_h, L.grid_w, L.X, L.Y, L.W)
+
+    def dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
+
+    for t in range(stepper.t):
+        kv.advance(t)
+        _, k, v = stepper.inputs(t)
+        kv.write_record(0, t, dev(k), dev(v))
+    t = stepper.t
+    q, k, v = stepper.inputs(t)
+    kv.advance(t)
+    o = torch.full((L.R, L.heads, L.d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    kv.write_attend(0, t, dev(q), dev(k), dev(v), o)
+    torch.cuda.synchronize()
+    kv.sync_status()
+    kd, vd = kv.kv_views(0)
+    kb = kd.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    vb = vd.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    ob = o.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    kv.close()
+    # the oracle's memory after the same frame (a copy: the stepper's own
+    # memory advances when it is timed)
+    import copy
+    mem = copy.deepcopy(stepper.mem)
+    mem.advance(t)
+    mem.write_record(0, t, k, v)
+    if not (np.array_equal(kb, mem.K[0]) and np.array_equal(vb, mem.V[0])):
+        raise RuntimeError("parity: the GPU buffers differ from the oracle's")
+    rng = np.random.default_rng(0x5EED)
+    rows = np.unique(np.concatenate([[0, L.HW - 1, L.HW, L.R - 1], rng.choice(L.R, 60, replace=False)]))
+    ref = attend_memory(mem, 0, q, rows=rows)
+    got = si.bf16_bits_to_f64(ob[rows])
+    if not np.isfinite(got).all():
+        raise RuntimeError("parity: non-finite attention output")
+    max_abs = float(np.abs(got - ref).max())
+    rel = float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
+    if max_abs > 2e-2 or rel > 5e-3:
+        raise RuntimeError(f"parity: attention max_abs {max_abs:.3e} rel_l2 {rel:.3e}")
+    return {"buffers": "bit-exact", "rows": int(len(rows)), "heads": L.heads,
+            "max_abs": round(max_abs, 6), "rel_l2": round(rel, 7), "frame": t,
+            "call": "wm_write_attend"}
+
+
+def cpu_baseline_and_parity(budget_s: float, torch=None, wm=None):
+    """The oracle timed on the host cores (served block, extrapolated to a
+    frame-step), one thread and the scaled memory as well; with ``wm`` given,
+    the GPU path is first checked against the oracle on the same inputs."""
+    stepper = OracleStepper()
+    parity = gpu_parity_on_stepper(stepper, torch, wm) if wm is not None else None
+    per_step, rows, t_attn, _ = stepper.step(budget_s)
     out = {"value": round(1.0 / per_step, 6), "unit": UNIT, "cores": _oracle_threads(),
            "kind": "oracle",
            "sample": f"{rows} query rows x 16 heads x 6528 keys of one block ({t_attn:.1f} s fp64 numpy), "
                      f"plus one eviction and one record write of that block's memory, "
                      f"extrapolated to 28 blocks x 1104 rows",
            "host_cpus": len(os.sched_getaffinity(0)), "cpu_model": _cpu_model()}
+    if parity is not None:
+        out["gpu_parity"] = parity
     small = max(0.5, budget_s / 4)
     try:
         from threadpoolctl import threadpool_limits
         with threadpool_limits(limits=1):
-            per1, rows1, t1 = OracleStepper().step(small)
+            per1, rows1, t1, _ = OracleStepper().step(small)
         out["one_thread"] = {"value": round(1.0 / per1, 6), "unit": UNIT, "cores": 1,
                              "sample": f"{rows1} query rows of one served block ({t1:.1f} s), "
                                        f"extrapolated the same way"}
@@ -763,7 +1008,7 @@ def cpu_baseline(budget_s: float):
     try:
         from oracle import Layout
         scaled = Layout(45, 80, 256, 2, 48, heads=24, d=128)
-        per_s, rows_s, t_s = OracleStepper(scaled, config_id=5, t_steady=60).step(small)
+        per_s, rows_s, t_s, _ = OracleStepper(scaled, config_id=5, t_steady=60).step(small)
         out["scaled"] = {"value": round(1.0 / per_s, 6), "unit": UNIT, "cores": _oracle_threads(),
                          "sample": f"{rows_s} query rows x 24 heads x {scaled.end(60)} keys of one "
                                    f"scaled block ({t_s:.1f} s), plus one eviction and one record "
@@ -771,6 +1016,11 @@ def cpu_baseline(budget_s: float):
     except Exception as e:
         out["scaled"] = {"error": f"{type(e).__name__}: {e}"}
     return out
+
+
+def cpu_baseline(budget_s: float):
+    """The CPU baseline without the GPU parity check."""
+    return cpu_baseline_and_parity(budget_s)
 
 
 def run_reference(args, world, rank):
@@ -783,12 +1033,12 @@ def run_reference(args, world, rank):
     for _ in range(args.warmup):
         stepper.step(budget)
     per = []
-    rows_total, attn_total = 0, 0.0
+    rows_total, spent_total = 0, 0.0
     for _ in range(args.steps):
-        s, rows, ta = stepper.step(budget)
+        s, rows, _, spent = stepper.step(budget)
         per.append(s)
         rows_total += rows
-        attn_total += ta
+        spent_total += spent
     total = sum(per)
     value = args.steps / total
     cores = _oracle_threads()
@@ -796,14 +1046,16 @@ def run_reference(args, world, rank):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": WORKLOAD, "blocks": BLOCKS, "heads": HEADS, "head_dim": D,
-                       "grid": f"{GH}x{GW}", "X": X, "Y": Y, "W": W, "queries": R, "keys": C,
-                       "parallelism": "host cores (fp64 oracle)"},
+            "config": config_dict(world),
+            "extrapolated": True,
+            "seconds_spent": round(spent_total, 2),
             "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
                              "cpu_model": _cpu_model(),
                              "sample": f"per step about {budget:.2f} s of query rows of one block "
                                        f"({rows_total} rows in all) plus one eviction and one record "
-                                       f"write, extrapolated to a full 28-block frame-step"},
+                                       f"write, extrapolated to a full 28-block frame-step; "
+                                       f"ms_per_step is that extrapolation, the timed steps took "
+                                       f"{spent_total:.1f} s of host time"},
             "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -818,9 +1070,18 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
-                    help="skip the secondary measurements (CUDA graphs, copy kernels' HBM "
-                         "throughput, batch of 8, scaled memory vs dense baseline)")
+                    help="skip the long runs and the secondary measurements (CUDA graphs, four-pass "
+                         "frame, copy kernels' HBM throughput, batch of 8, scaled memory vs dense)")
+    ap.add_argument("--ncu-csv", help="summarise this ncu --csv capture and exit (no GPU)")
+    ap.add_argument("--ncu-out", help="JSON file the summary is written to")
+    ap.add_argument("--ncu-cmd", default="", help="the ncu command line, recorded in the summary")
     args = ap.parse_args()
+    if args.ncu_csv:
+        summary = summarize_ncu_csv(args.ncu_csv, args.ncu_cmd)
+        with open(args.ncu_out, "w") as f:
+            json.dump(summary, f, indent=1)
+            f.write("\n")
+        return
     args.warmup = max(3, args.warmup)      # at least 3 untimed warm-up steps
     world, rank, local = dist_setup()
     if args.impl == "reference":

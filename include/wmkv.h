@@ -72,7 +72,12 @@ enum {
 };
 
 /* Create the memory of one session: `blocks` per-block K/V buffer pairs on the
- * current CUDA device, zero-filled, in one allocation of
+ * current CUDA device.  Defined by the model card, section "One buffer, no
+ * mask" (one preallocated buffer per block, | Z0 | RAW (Y+1) records | SUM
+ * (W-Y) x X summary rows |, capacity C = R*(Y+2) + X*(W-Y) rows: 6,528 at the
+ * served 24x42 grid with X = 96, Y = 2, W = 24) and section "A frame is a
+ * record" (R = grid_h*grid_w raw rows followed by X summary rows).
+ * Buffers are zero-filled, in one allocation of
  * blocks * 2 * C * heads * d * 2 bytes (block b's K buffer first, then its V).
  * Requirements: blocks >= 1, heads >= 1, d in {64, 128}, grid_h >= 1,
  * grid_w >= 1, X >= 1, 0 <= Y <= W (W == Y gives an empty SUM region).
@@ -98,7 +103,12 @@ WM_API int wm_advance(wm_kvbuf* h, int64_t t, wm_stream_t stream);
 WM_API int wm_write_record(wm_kvbuf* h, int block, int64_t t, const void* K, const void* V,
                     wm_stream_t stream);
 
-/* Dense unmasked attention of frame t's queries over buffer[0:end] of `block`:
+/* Dense unmasked attention of frame t's queries over buffer[0:end] of `block`
+ * (model card, section "One buffer, no mask": every query of the frame being
+ * generated attends to the whole filled prefix of its block's buffer, with no
+ * mask, because the buffer holds exactly the keys the frame may see; section
+ * "The rest of the model", Attention kernels, for the ordinary 1/sqrt(d)
+ * softmax of the kernels it names):
  *   O[i,h,:] = sum_j softmax_j(Q[i,h,:] . K[j,h,:] / sqrt(d)) V[j,h,:],  j < end.
  * Q and O are device arrays [R, heads, d] bf16.  Scores, softmax and the
  * accumulation are fp32 on the tensor cores (P rounded to bf16 for P.V); O is
@@ -107,7 +117,9 @@ WM_API int wm_write_record(wm_kvbuf* h, int block, int64_t t, const void* K, con
 WM_API int wm_attend(wm_kvbuf* h, int block, const void* Q, void* O, wm_stream_t stream);
 
 /* wm_write_record followed by wm_attend for the same block and frame, in one
- * launch where the head dimension allows (d = 64): the attention reads the
+ * launch where the head dimension allows (d = 64).  The two steps are the
+ * model card's (sections "A frame is a record" and "One buffer, no mask");
+ * doing them in one launch is this library's: the attention reads the
  * keys before and after the record's slot from the buffer and the record
  * itself from K/V (softmax attention does not depend on the order of the
  * keys), while the same launch copies K/V into the slot.  Results and buffer
@@ -154,6 +166,20 @@ WM_API int wm_kv_ptrs(const wm_kvbuf* h, int block, void** K, void** V);
  * WM_ERR_CUDA if the synchronisation itself failed, else WM_OK. */
 WM_API int wm_sync_status(wm_kvbuf* h);
 
+/* Bound, in SM clock cycles, on each wait inside this handle's attention
+ * launches (wm_attend, wm_write_attend) for work another part of the same
+ * launch produces (tensor loads, tensor-core results, softmax tiles).  The
+ * default, 4e9 cycles (about 2 s at the 1.965 GHz maximum clock), is far above
+ * any wait of a healthy launch.  A launch that runs out of it finishes the
+ * copies and tensor-core work it started, releases its tensor memory, exits,
+ * and leaves WM_ERR_TIMEOUT for wm_sync_status; its outputs, and a slot that a
+ * wm_write_attend in it was writing, are then undefined until written again.
+ * A smaller bound exercises that path: 0 makes the first wait that is not
+ * already satisfied give up.  The page has no counterpart: this is the
+ * library's guard against a launch that would otherwise never end.
+ * Returns WM_ERR_INVALID_ARG for a NULL handle. */
+WM_API int wm_set_wait_limit(wm_kvbuf* h, uint64_t cycles);
+
 /* Static description of an error code. */
 WM_API const char* wm_strerror(int code);
 /* Text of the last CUDA error seen by this thread in a wm_* call ("" if none). */
@@ -167,13 +193,15 @@ WM_API int wm_layout_sum_slot(int Y, int W, int64_t f);
 /* First row of frame t's record (Z0 for t = 0, its RAW slot otherwise). */
 WM_API int64_t wm_layout_record_row(int grid_h, int grid_w, int X, int Y, int64_t t);
 
-/* Dense attention with no frame memory.  The page contrasts the 6,528 keys
- * of the served buffer with the 26,208 the same span would need at full
- * resolution; this call runs that full-resolution comparison point:
+/* Dense attention with no frame memory.  The model card (section "One
+ * buffer, no mask") contrasts the 6,528 keys of the served buffer with the
+ * 26,208 the same span would need at full resolution; this call runs that
+ * full-resolution comparison point:
  *   O[i,h,:] = sum_j softmax_j(Q[i,h,:] . K[j,h,:] / sqrt(d)) V[j,h,:],  j < Lk,
  * Q/O device [Lq, heads, d], K/V device [Lk, heads, d], all bf16, same
  * kernel and numerics as wm_attend.  Lq >= 1, Lk >= 1, d in {64, 128}.
- * `dev_status` is an optional device int (NULL to skip) that the kernel sets
+ * Beyond the page's statement of the operation, the call takes a stream and
+ * `dev_status`, an optional device int (NULL to skip) that the kernel sets
  * to 1 if it gives up a bounded wait (about 2 s); it is not touched
  * otherwise, so the caller zeroes it beforehand and reads it after the
  * stream has reached the launch.

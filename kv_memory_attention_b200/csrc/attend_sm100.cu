@@ -37,7 +37,7 @@
 // The two warpgroups' partial results (m, l, O) are merged row by row at the
 // end and stored as bf16.
 //
-// Every mbarrier wait is bounded (about 2 s); a CTA that gives up sets a shared
+// Every mbarrier wait is bounded (by default about 2 s); a CTA that gives up sets a shared
 // abort flag, records DEV_TIMEOUT in the caller's status word, drains what it
 // issued, frees TMEM and exits.
 #include <cuda.h>
@@ -64,9 +64,10 @@ constexpr int SOFTMAX_REGS = 224;
 constexpr int CONTROL_REGS = 56;
 static_assert(256 * SOFTMAX_REGS + 128 * CONTROL_REGS <= NUM_THREADS * LAUNCH_REGS,
               "register split exceeds the launch budget");
-// Bounded waits, in SM cycles: about 2 s (0.2 s for the drain after a
-// timeout) at the 1.965 GHz maximum clock, longer at lower clocks.
-constexpr uint64_t WAIT_LIMIT_CYCLES = 4000000000ull;
+// Bounded waits: each wait gives up after AttendParams::wait_limit SM cycles
+// (by default about 2 s at the 1.965 GHz maximum clock, longer at lower
+// clocks); the drain after a timeout waits up to 0.2 s per operation,
+// whatever the limit.
 constexpr uint64_t DRAIN_LIMIT_CYCLES = 400000000ull;
 #ifndef WMKV_RESCALE_THRESHOLD
 #define WMKV_RESCALE_THRESHOLD 8.0f
@@ -175,6 +176,7 @@ struct AttendParams {
   const uint4* copy_src[2];
   uint4* copy_dst[2];
   int64_t copy_n16;
+  uint64_t wait_limit;  // SM cycles per bounded wait
 };
 
 // Segment and row of key tile j, and how many of its 128 rows are keys.
@@ -316,11 +318,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
             bulk_load(sbase + C::COPY_OFF + t * C::COPY_CHUNK_BYTES, p.copy_src[t] + u, bytes,
                       bar(C::B_COPY + t));
           }
-          for (int t = 0; t < 2; ++t) {
-            if (!mbar_wait_bounded(bar(C::B_COPY + t), cph, abort_flag, WAIT_LIMIT_CYCLES)) break;
-            bulk_store(p.copy_dst[t] + u, sbase + C::COPY_OFF + t * C::COPY_CHUNK_BYTES, bytes);
+          int landed = 0;
+          for (; landed < 2; ++landed) {
+            if (!mbar_wait_bounded(bar(C::B_COPY + landed), cph, abort_flag, p.wait_limit)) break;
+            bulk_store(p.copy_dst[landed] + u, sbase + C::COPY_OFF + landed * C::COPY_CHUNK_BYTES,
+                       bytes);
           }
           bulk_commit();
+          if (landed < 2) {
+            // gave up: let the staging loads still in flight land before the
+            // CTA can exit (their shared memory goes to the next CTA)
+            volatile int no_abort = 0;
+            for (int t = landed; t < 2; ++t)
+              mbar_wait_bounded(bar(C::B_COPY + t), cph, &no_abort, DRAIN_LIMIT_CYCLES);
+            break;
+          }
           cph ^= 1;
         }
       };
@@ -334,7 +346,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
         if (i < nkv) {
           const int st = i % C::NK;
           if (i >= C::NK && !mbar_wait_bounded(bar(C::B_KEMPTY + st), ((i / C::NK) - 1) & 1,
-                                               abort_flag, WAIT_LIMIT_CYCLES))
+                                               abort_flag, p.wait_limit))
             break;
           const TileLoc tl = tile_loc(p, i);
           mbar_expect_tx(bar(C::B_KFULL + st), C::TILE_BYTES);
@@ -347,7 +359,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
         if (jv >= 0 && jv < nkv) {
           const int st = jv % C::NV;
           if (jv >= C::NV && !mbar_wait_bounded(bar(C::B_VEMPTY + st), ((jv / C::NV) - 1) & 1,
-                                                abort_flag, WAIT_LIMIT_CYCLES))
+                                                abort_flag, p.wait_limit))
             break;
           const TileLoc tl = tile_loc(p, jv);
           mbar_expect_tx(bar(C::B_VFULL + st), C::TILE_BYTES);
@@ -362,6 +374,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
       if (*abort_flag) {
         // Let the copies this thread started land before the CTA exits.
         volatile int no_abort = 0;
+        mbar_wait_bounded(bar(C::B_Q), 0, &no_abort, DRAIN_LIMIT_CYCLES);
         for (int i = k_issued - C::NK < 0 ? 0 : k_issued - C::NK; i < k_issued; ++i)
           mbar_wait_bounded(bar(C::B_KFULL + i % C::NK), (i / C::NK) & 1, &no_abort,
                             DRAIN_LIMIT_CYCLES);
@@ -391,9 +404,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
           const uint64_t dk0 = sdesc_sw128(sbase + C::K_OFF, 16, 1024);
           const uint64_t dv0 = sdesc_sw128(sbase + C::V_OFF, C::SUB_BYTES, 1024);
           uint32_t k_st = 0, k_ph = 0, v_st = 0, v_ph = 0, pf_ph = 0;
-          ok = mbar_spin_bounded(bar(C::B_Q), 0, abort_flag, WAIT_LIMIT_CYCLES);
+          ok = mbar_spin_bounded(bar(C::B_Q), 0, abort_flag, p.wait_limit);
           auto do_s = [&](int g) -> bool {
-            if (!mbar_spin_bounded(bar(C::B_KFULL + k_st), k_ph, abort_flag, WAIT_LIMIT_CYCLES))
+            if (!mbar_spin_bounded(bar(C::B_KFULL + k_st), k_ph, abort_flag, p.wait_limit))
               return false;
             tc_fence_after();
             issue_s<D>(dq, dk0 + k_st * TILE16, tmem + (g ? C::S_COL1 : C::S_COL0));
@@ -406,8 +419,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
           for (int j = 0; ok && j < nkv; ++j) {
             const int g = j & 1;
             if (!mbar_wait_bounded(bar(C::B_PFULL + g), (pf_ph >> g) & 1, abort_flag,
-                                   WAIT_LIMIT_CYCLES) ||
-                !mbar_spin_bounded(bar(C::B_VFULL + v_st), v_ph, abort_flag, WAIT_LIMIT_CYCLES)) {
+                                   p.wait_limit) ||
+                !mbar_spin_bounded(bar(C::B_VFULL + v_st), v_ph, abort_flag, p.wait_limit)) {
               ok = false;
               break;
             }
@@ -431,7 +444,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
         const uint64_t dk0 = sdesc_sw128(sbase + C::K_OFF, 16, 1024);
         uint32_t k_st = 0, k_ph = 0;  // ring slot / phase of the next K tile
         uint32_t fr_ph = 0;           // bit g: phase of the barrier that frees S_g
-        ok = mbar_spin_bounded(bar(C::B_Q), 0, abort_flag, WAIT_LIMIT_CYCLES);
+        ok = mbar_spin_bounded(bar(C::B_Q), 0, abort_flag, p.wait_limit);
         for (int j = 0; ok && j < nkv; ++j) {
           const int g = j & 1;
           if (j >= 2) {
@@ -439,13 +452,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
             // own columns) or once P_{j-2}.V_{j-2} has completed (d = 128: P
             // overwrote S_{j-2})
             const int fb = C::P_SEP ? C::B_SFREE + g : C::B_ODONE + g;
-            if (!mbar_wait_bounded(bar(fb), (fr_ph >> g) & 1, abort_flag, WAIT_LIMIT_CYCLES)) {
+            if (!mbar_wait_bounded(bar(fb), (fr_ph >> g) & 1, abort_flag, p.wait_limit)) {
               ok = false;
               break;
             }
             fr_ph ^= 1u << g;
           }
-          if (!mbar_spin_bounded(bar(C::B_KFULL + k_st), k_ph, abort_flag, WAIT_LIMIT_CYCLES)) {
+          if (!mbar_spin_bounded(bar(C::B_KFULL + k_st), k_ph, abort_flag, p.wait_limit)) {
             ok = false;
             break;
           }
@@ -466,8 +479,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
         for (int j = g; ok && j < nkv; j += 2) {
           const int v_st = j % C::NV;
           const uint32_t v_ph = (j / C::NV) & 1;
-          if (!mbar_wait_bounded(bar(C::B_PFULL + g), pf_ph, abort_flag, WAIT_LIMIT_CYCLES) ||
-              !mbar_spin_bounded(bar(C::B_VFULL + v_st), v_ph, abort_flag, WAIT_LIMIT_CYCLES)) {
+          if (!mbar_wait_bounded(bar(C::B_PFULL + g), pf_ph, abort_flag, p.wait_limit) ||
+              !mbar_spin_bounded(bar(C::B_VFULL + v_st), v_ph, abort_flag, p.wait_limit)) {
             ok = false;
             break;
           }
@@ -505,7 +518,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
     bool ok = true;
     int n = 0;
     for (int j = wg; j < nkv; j += 2, ++n) {
-      ok = mbar_wait_bounded(bar(C::B_SFULL + wg), n & 1, abort_flag, WAIT_LIMIT_CYCLES);
+      ok = mbar_wait_bounded(bar(C::B_SFULL + wg), n & 1, abort_flag, p.wait_limit);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
@@ -586,7 +599,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
       l_run = l_run * alpha + (a_lo + a_hi);
       if (n > 0) {
         // P.V of this warpgroup's previous tile has finished: O is stable, P is free
-        ok = mbar_wait_bounded(bar(C::B_ODONE + wg), (n - 1) & 1, abort_flag, WAIT_LIMIT_CYCLES);
+        ok = mbar_wait_bounded(bar(C::B_ODONE + wg), (n - 1) & 1, abort_flag, p.wait_limit);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
@@ -618,7 +631,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
     }
     // all P.V products must have landed before O is read
     if (ok) {
-      ok = mbar_wait_bounded(bar(C::B_OFINAL), 0, abort_flag, WAIT_LIMIT_CYCLES);
+      ok = mbar_wait_bounded(bar(C::B_OFINAL), 0, abort_flag, p.wait_limit);
       ok = __all_sync(0xffffffffu, ok);
     }
     tc_fence_after();
@@ -738,7 +751,7 @@ bool attend_copies_in_kernel(int d) { return Cfg<64>::COPY_IN_KERNEL && d == 64;
 
 cudaError_t launch_attend(const void* q, void* o, int64_t lq, const KVSegment* segs, int nseg,
                           int heads, int d, int* status, const RecordCopy* copy,
-                          cudaStream_t stream) {
+                          unsigned long long wait_limit, cudaStream_t stream) {
   if (nseg < 1 || nseg > MAX_SEGS) return cudaErrorInvalidValue;
   AttendParams prm = {};
   if (!encode_rows_map(&prm.tm_q, q, lq, heads, d)) return cudaErrorInvalidValue;
@@ -758,6 +771,7 @@ cudaError_t launch_attend(const void* q, void* o, int64_t lq, const KVSegment* s
   prm.heads = heads;
   prm.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
   prm.status = status;
+  prm.wait_limit = wait_limit;
   if (copy && copy->n16 > 0) {
     if (!attend_copies_in_kernel(d)) return cudaErrorInvalidValue;
     prm.copy_src[0] = static_cast<const uint4*>(copy->k_src);

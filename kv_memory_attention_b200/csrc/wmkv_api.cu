@@ -38,6 +38,7 @@ struct wm_kvbuf {
   std::vector<double> theta;   // per dimension pair, radians per frame (0: not temporal)
   int gap_trigger = 5, gap_target = 1;
   int64_t z0_pos = 0;          // temporal position of the start image
+  unsigned long long wait_limit = wmkv::DEFAULT_WAIT_LIMIT_CYCLES;  // attention launches
 };
 
 namespace {
@@ -256,8 +257,14 @@ int wm_attend(wm_kvbuf* h, int block, const void* Q, void* O, wm_stream_t stream
   const uint8_t* vbuf = kbuf + h->tensor_bytes;
   const wmkv::KVSegment seg = {kbuf, vbuf, end};
   cudaError_t e = wmkv::launch_attend(Q, O, h->R, &seg, 1, h->heads, h->d, h->status, nullptr,
-                                      reinterpret_cast<cudaStream_t>(stream));
+                                      h->wait_limit, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
+  return WM_OK;
+}
+
+int wm_set_wait_limit(wm_kvbuf* h, uint64_t cycles) {
+  if (!h) return WM_ERR_INVALID_ARG;
+  h->wait_limit = cycles;
   return WM_OK;
 }
 
@@ -287,12 +294,14 @@ int wm_write_attend(wm_kvbuf* h, int block, int64_t t, const void* Q, const void
       segs[nseg++] = {kbuf + after * h->row_bytes, vbuf + after * h->row_bytes, end - after};
     segs[nseg++] = {K, V, h->R};
     const wmkv::RecordCopy cp = {K, V, kslot, vslot, n16};
-    e = wmkv::launch_attend(Q, O, h->R, segs, nseg, h->heads, h->d, h->status, &cp, s);
+    e = wmkv::launch_attend(Q, O, h->R, segs, nseg, h->heads, h->d, h->status, &cp, h->wait_limit,
+                            s);
   } else {
     e = wmkv::launch_copy_pair(K, V, kslot, vslot, n16, s);
     const wmkv::KVSegment seg = {kbuf, vbuf, end};
     if (e == cudaSuccess)
-      e = wmkv::launch_attend(Q, O, h->R, &seg, 1, h->heads, h->d, h->status, nullptr, s);
+      e = wmkv::launch_attend(Q, O, h->R, &seg, 1, h->heads, h->d, h->status, nullptr,
+                              h->wait_limit, s);
   }
   if (e != cudaSuccess) return cuda_fail(e);
   h->written[block] = t;
@@ -373,6 +382,7 @@ int wm_attend_dense(const void* Q, const void* K, const void* V, void* O, int64_
   if ((Lq + 127) / 128 > 0x7FFFFFFF || heads > 65535) return WM_ERR_INVALID_ARG;
   const wmkv::KVSegment seg = {K, V, Lk};
   cudaError_t e = wmkv::launch_attend(Q, O, Lq, &seg, 1, heads, d, dev_status, nullptr,
+                                      wmkv::DEFAULT_WAIT_LIMIT_CYCLES,
                                       reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
   return WM_OK;

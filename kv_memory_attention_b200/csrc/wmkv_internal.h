@@ -56,9 +56,13 @@ struct RecordCopy {
 // (softmax over all of them together), O [lq, heads, d]: see attend_sm100.cu.
 // `copy` (may be null) is performed by the same launch; only supported where
 // attend_copies_in_kernel(d).  Returns a cudaError_t from encoding/launching.
+// Bound on each wait inside an attention launch, in SM cycles (about 2 s at
+// the 1.965 GHz maximum clock).
+constexpr unsigned long long DEFAULT_WAIT_LIMIT_CYCLES = 4000000000ull;
+
 cudaError_t launch_attend(const void* q, void* o, int64_t lq, const KVSegment* segs, int nseg,
                           int heads, int d, int* status, const RecordCopy* copy,
-                          cudaStream_t stream);
+                          unsigned long long wait_limit, cudaStream_t stream);
 bool attend_copies_in_kernel(int d);
 
 // Copy `n16` 16-byte chunks of a and b (two independent arrays) in one launch.

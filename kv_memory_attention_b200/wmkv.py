@@ -43,6 +43,7 @@ SIGNATURES = {
     "wm_sum_slot": (_c_int, [_vp, _c_i64]),
     "wm_kv_ptrs": (_c_int, [_vp, _c_int, ctypes.POINTER(_vp), ctypes.POINTER(_vp)]),
     "wm_sync_status": (_c_int, [_vp]),
+    "wm_set_wait_limit": (_c_int, [_vp, ctypes.c_uint64]),
     "wm_strerror": (ctypes.c_char_p, [_c_int]),
     "wm_last_cuda_error": (ctypes.c_char_p, []),
     "wm_layout_capacity": (_c_i64, [_c_int, _c_int, _c_int, _c_int, _c_int]),
@@ -179,6 +180,13 @@ def wm_sync_status(h: int) -> None:
     _check(LIB.wm_sync_status(h), "wm_sync_status")
 
 
+def wm_set_wait_limit(h: int, cycles: int) -> None:
+    _check(LIB.wm_set_wait_limit(h, cycles), "wm_set_wait_limit")
+
+
+DEFAULT_WAIT_LIMIT_CYCLES = 4_000_000_000
+
+
 def wm_strerror(code: int) -> str:
     return LIB.wm_strerror(code).decode()
 
@@ -261,6 +269,9 @@ class KVMemory:
 
     def sync_status(self):
         wm_sync_status(self.h)
+
+    def set_wait_limit(self, cycles):
+        wm_set_wait_limit(self.h, cycles)
 
     def kv_views(self, block):
         import torch

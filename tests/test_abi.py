@@ -87,6 +87,7 @@ def test_null_handle_and_pointer_errors(wm):
     assert lib.wm_write_record(None, 0, 0, 16, 16, None) == wm.WM_ERR_INVALID_ARG
     assert lib.wm_attend(None, 0, 16, 16, None) == wm.WM_ERR_INVALID_ARG
     assert lib.wm_sync_status(None) == wm.WM_ERR_INVALID_ARG
+    assert lib.wm_set_wait_limit(None, 5) == wm.WM_ERR_INVALID_ARG
     assert lib.wm_kvbuf_destroy(None) == wm.WM_ERR_INVALID_ARG
     assert lib.wm_end(None) == -1
     # dense: misaligned / null pointers and bad sizes never reach the device
