@@ -9,9 +9,11 @@ library.
 from .kvmemory import (Layout, FrameMemory, attend, attend_bits, attend_memory,
                        softmax_weights, visible_history_mask, masked_history_attend,
                        rotation_cos_sin, rotate_pairs_f64, rotate_keys_bf16, sink_shift,
-                       TINY, SERVED, SERVED_W16, SCALED)
+                       E4M3_MAX, E4M3_NAN, e4m3_decode, e4m3_encode, quantize_e4m3,
+                       dequantize_e4m3, TINY, SERVED, SERVED_W16, SCALED)
 
 __all__ = ["Layout", "FrameMemory", "attend", "attend_bits", "attend_memory",
            "softmax_weights", "visible_history_mask", "masked_history_attend",
            "rotation_cos_sin", "rotate_pairs_f64", "rotate_keys_bf16", "sink_shift",
-           "TINY", "SERVED", "SERVED_W16", "SCALED"]
+           "E4M3_MAX", "E4M3_NAN", "e4m3_decode", "e4m3_encode", "quantize_e4m3",
+           "dequantize_e4m3", "TINY", "SERVED", "SERVED_W16", "SCALED"]

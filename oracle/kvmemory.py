@@ -54,6 +54,16 @@ notes of the repository):
      sum rounded to float32, c and s the float32 cosine and sine) and rounded
      to bfloat16: the page gives neither the frequencies nor the precision,
      so the frequencies are a parameter and the precision is the kernel's.
+  R7 (FP8 buffer; the page of another system, "commaai/worldmodel-4B", README,
+     says only that its checkpoint keeps FP8 KV caches) the buffer may store
+     K and V as OCP FP8 E4M3 codes (1 sign, 4 exponent bits with bias 7, 3
+     mantissa bits, subnormals, no infinities, S.1111.111 = NaN, largest
+     finite value 448).  Each (block, head) has one float32 scale for K and
+     one for V, fixed when the buffer is created.  A stored code is the
+     float32 quotient x / scale rounded to nearest, ties to even, and
+     saturated to +-448 (NaN stays NaN); a code means code_value * scale.
+     Eviction moves codes.  Attention is the same softmax over the dequantised
+     values.  The streaming sink is not defined for this format.
 """
 from __future__ import annotations
 
@@ -196,6 +206,67 @@ def sink_shift(layout: "Layout", t: int, z0_pos: int, trigger: int = 5, target: 
 
 
 # ---------------------------------------------------------------------------
+# FP8 E4M3 codes (reading R7)
+# ---------------------------------------------------------------------------
+
+E4M3_MAX = 448.0          # 1.75 * 2^8, the largest finite E4M3 value
+E4M3_NAN = 0x7F           # the code a NaN input gets
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """Value of each E4M3 code as float64: sign, 4-bit exponent (bias 7) and
+    3-bit mantissa; exponent field 0 holds the subnormals m/8 * 2^-6; the
+    all-ones exponent with all-ones mantissa is NaN."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    val = sign * mag
+    return np.where((e == 15) & ((c & 7) == 7), np.nan, val)
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """E4M3 code of each value: nearest representable value, ties to the even
+    mantissa; magnitudes of 448 and above saturate to 448; NaN -> E4M3_NAN."""
+    v = np.asarray(x, dtype=np.float64)
+    neg = np.signbit(v)
+    a = np.abs(v)
+    nan = np.isnan(a)
+    a = np.where(nan, 0.0, a)
+    # subnormal range, a < 2^-6: units of 2^-9 (the value 8 * 2^-9 is the
+    # smallest normal, code 0x08, which the same formula produces)
+    sub = np.rint(np.where(a < 2.0 ** -6, a, 0.0) / 2.0 ** -9)
+    # normal range: a = (1 + f) * 2^e with f in [0, 1)
+    mant, ex = np.frexp(np.where((a > 0) & (a < E4M3_MAX), a, 1.0))   # a = mant * 2^ex
+    e = ex - 1
+    m = np.rint((mant * 2.0 - 1.0) * 8.0)               # 3-bit mantissa, half to even
+    carry = m == 8
+    e = np.where(carry, e + 1, e)
+    m = np.where(carry, 0, m)
+    normal = ((e + 7) << 3) | m.astype(np.int64)
+    code = np.where(a < 2.0 ** -6, sub.astype(np.int64), normal)
+    code = np.where(a >= E4M3_MAX, 0x7E, code)
+    code = code | np.where(neg, 0x80, 0)
+    code = np.where(nan, E4M3_NAN, code)
+    return code.astype(np.uint8)
+
+
+def quantize_e4m3(bits: np.ndarray, scale) -> np.ndarray:
+    """bf16 bit patterns ``[rows, heads, d]`` -> E4M3 codes with one float32
+    scale per head: code = e4m3(float32(x) / scale), the division in float32."""
+    x = si.bf16_bits_to_f32(bits)
+    s = np.asarray(scale, dtype=np.float32).reshape(1, -1, 1)
+    return e4m3_encode(np.divide(x, s, dtype=np.float32))
+
+
+def dequantize_e4m3(codes: np.ndarray, scale) -> np.ndarray:
+    """E4M3 codes ``[rows, heads, d]`` -> code value * scale (per head), float64 (exact)."""
+    s = np.asarray(scale, dtype=np.float32).astype(np.float64).reshape(1, -1, 1)
+    return e4m3_decode(codes) * s
+
+
+# ---------------------------------------------------------------------------
 # The memory: a host mirror updated by the page's rules
 # ---------------------------------------------------------------------------
 
@@ -219,12 +290,21 @@ class FrameMemory:
     raw_tag: list = field(init=False)        # frame id held by each RAW slot
     sum_tag: list = field(init=False)        # frame id whose summary each SUM slot holds
     written: set = field(init=False)         # blocks written at the current t
+    kv_format: str = "bf16"                  # "bf16" bit patterns or "e4m3" codes (R7)
+    k_scale: object = None                   # e4m3: float32 [blocks, heads]
+    v_scale: object = None
 
     def __post_init__(self):
         L = self.layout
         shape = (self.blocks, L.C, L.heads, L.d)
-        self.K = np.zeros(shape, dtype=np.uint16)
-        self.V = np.zeros(shape, dtype=np.uint16)
+        if self.kv_format not in ("bf16", "e4m3"):
+            raise ValueError(self.kv_format)
+        store = np.uint8 if self.kv_format == "e4m3" else np.uint16
+        if self.kv_format == "e4m3":
+            self.k_scale = np.asarray(self.k_scale, np.float32).reshape(self.blocks, L.heads)
+            self.v_scale = np.asarray(self.v_scale, np.float32).reshape(self.blocks, L.heads)
+        self.K = np.zeros(shape, dtype=store)
+        self.V = np.zeros(shape, dtype=store)
         self.records = {}
         self.raw_tag = [None] * (L.Y + 1)
         self.sum_tag = [None] * max(L.W - L.Y, 0)
@@ -252,6 +332,8 @@ class FrameMemory:
             self.V[:, d0:d1] = self.V[:, src0:r1]
             self.sum_tag[u] = f
         if self.sink_theta is not None:
+            if self.kv_format != "bf16":
+                raise ValueError("the streaming sink is defined for bf16 buffers only")
             shift = sink_shift(L, t, self.z0_pos)
             if shift:
                 self.K[:, :L.R] = rotate_keys_bf16(self.K[:, :L.R], self.sink_theta, shift)
@@ -269,6 +351,9 @@ class FrameMemory:
         if t != self.t:
             raise ValueError(f"write_record at t={t}, current frame {self.t}")
         assert k.shape == v.shape == (L.R, L.heads, L.d)
+        if self.kv_format == "e4m3":
+            k = quantize_e4m3(k, self.k_scale[block])
+            v = quantize_e4m3(v, self.v_scale[block])
         r0, r1 = L.record_rows(t)
         self.K[block, r0:r1] = k
         self.V[block, r0:r1] = v
@@ -279,8 +364,11 @@ class FrameMemory:
         self.written.add(block)
 
     def prefix(self, block: int):
-        """K, V of buffer[0:end] as fp64 arrays ``[end, heads, d]``."""
+        """K, V of buffer[0:end] as fp64 arrays ``[end, heads, d]`` (dequantised for e4m3)."""
         e = self.end()
+        if self.kv_format == "e4m3":
+            return (dequantize_e4m3(self.K[block, :e], self.k_scale[block]),
+                    dequantize_e4m3(self.V[block, :e], self.v_scale[block]))
         return si.bf16_bits_to_f64(self.K[block, :e]), si.bf16_bits_to_f64(self.V[block, :e])
 
     def check_against_records(self) -> None:

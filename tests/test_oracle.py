@@ -186,6 +186,16 @@ def test_weights_sum_to_one():
     assert (w >= 0).all()
 
 
+def test_weights_two_keys_logistic():
+    """softmax_weights of two keys: logistic((s0 - s1) / sqrt(d)); pins its scale."""
+    d = 64
+    q = np.zeros((1, 1, d)); q[0, 0, 3] = 2.0
+    k = np.zeros((2, 1, d)); k[0, 0, 3] = 5.0; k[1, 0, 3] = -3.0
+    w = softmax_weights(q, k)
+    w0 = 1.0 / (1.0 + np.exp(-(2.0 * 5.0 - 2.0 * -3.0) / 8.0))
+    np.testing.assert_allclose(w[0, 0], [w0, 1.0 - w0], rtol=0, atol=1e-15)
+
+
 def test_constant_values_give_constant_output():
     rng = np.random.default_rng(3)
     q, k = rng.standard_normal((5, 2, 16)), rng.standard_normal((40, 2, 16))
