@@ -112,9 +112,12 @@ def source_digest() -> str:
 
 # ---------------------------------------------------------------- ncu summaries
 
-_TIME_UNITS = {"nsecond": 1e-3, "usecond": 1.0, "msecond": 1e3, "second": 1e6}
+_TIME_UNITS = {"nsecond": 1e-3, "usecond": 1.0, "msecond": 1e3, "second": 1e6,
+               "ns": 1e-3, "us": 1.0, "ms": 1e3, "s": 1e6}
 _BYTE_UNITS = {"byte": 1.0, "kbyte": 1e3, "mbyte": 1e6, "gbyte": 1e9,
-               "kibyte": 1024.0, "mibyte": 1024.0 ** 2, "gibyte": 1024.0 ** 3}
+               "kibyte": 1024.0, "mibyte": 1024.0 ** 2, "gibyte": 1024.0 ** 3,
+               "b": 1.0, "kb": 1e3, "mb": 1e6, "gb": 1e9, "kib": 1024.0, "mib": 1024.0 ** 2,
+               "gib": 1024.0 ** 3}
 
 
 def _kernel_short_name(name: str) -> str:
@@ -832,6 +835,38 @@ def extra_scaled(torch, wm, device, pk, steps=3):
                    "the full history; per-block inputs are windows of one random pool per tensor"}
 
 
+def extra_fp8(torch, wm, Q, K, V, O, steps=50):
+    """The served frame-step on an FP8 (E4M3) memory: same inputs, one scale of
+    1/64 for every (block, head) of K and V; each write_attend is three launches
+    (quantise the record into its slot, widen the block's codes to bf16, attend)."""
+    n = BLOCKS * HEADS
+    kv8 = wm.KVMemory(BLOCKS, HEADS, D, GH, GW, X, Y, W, kv_format="e4m3",
+                      k_scale=[1 / 64] * n, v_scale=[1 / 64] * n)
+    for t in range(T_STEADY):
+        kv8.advance(t)
+        for b in range(BLOCKS):
+            kv8.write_record(b, t, K[b], V[b])
+    t = T_STEADY
+
+    def step():
+        nonlocal t
+        kv8.advance(t)
+        for b in range(BLOCKS):
+            kv8.write_attend(b, t, Q[b], K[b], V[b], O[b])
+        t += 1
+
+    for _ in range(3):
+        step()
+    ms = _timed(torch, step, steps)
+    kv8.sync_status()
+    kv8.close()
+    return {"value": round(1e3 / ms, 3), "unit": UNIT, "ms_per_step": round(ms, 4), "steps": steps,
+            "launches_per_step": 1 + 3 * BLOCKS,
+            "buffer_bytes": 2 * BLOCKS * C * HEADS * D,
+            "tflops_per_step": round(BLOCKS * ATTN_FLOP / (ms * 1e-3) / 1e12, 1),
+            "how": "advance + 28 x write_attend on an E4M3 memory (quantise, widen, attend)"}
+
+
 def run_extras(torch, wm, device, kv, t, Q, K, V, O, window):
     """All secondary measurements; a section that fails reports its error."""
     pk = peaks()
@@ -840,6 +875,7 @@ def run_extras(torch, wm, device, kv, t, Q, K, V, O, window):
                      ("four_pass_frame", lambda: extra_four_pass(torch, kv, t, Q, K, V, O)),
                      ("copy_kernels", lambda: extra_copies(torch, kv, t, K, V, pk["hbm"])),
                      ("batch8", lambda: (extra_batch(torch, wm, window, device), t)),
+                     ("fp8_buffer", lambda: (extra_fp8(torch, wm, Q, K, V, O), t)),
                      ("scaled_vs_dense", lambda: (extra_scaled(torch, wm, device, pk), t))):
         try:
             out[name], t = fn()

@@ -86,6 +86,34 @@ enum {
 WM_API int wm_kvbuf_create(wm_kvbuf** out, int blocks, int heads, int d, int grid_h, int grid_w, int X,
                     int Y, int W);
 
+/* Storage formats of a session's buffers (wm_kv_format). */
+enum { WM_KV_BF16 = 0, WM_KV_E4M3 = 1 };
+
+/* The same memory with K and V stored as FP8 E4M3 codes, one byte per value.
+ * The page of another system ("commaai/worldmodel-4B", README) says its
+ * checkpoint keeps FP8 KV caches and names no scaling; this library reads
+ * that as OCP FP8 E4M3 (sign, 4 exponent bits with bias 7, 3 mantissa bits,
+ * subnormals, no infinities, largest finite 448) with one float32 scale per
+ * (block, head) for K and one for V: k_scale[block * heads + h], likewise
+ * v_scale, host arrays of blocks * heads positive finite floats, copied.
+ * wm_write_record / wm_write_attend store code = E4M3(x / scale) (float32
+ * division, round to nearest even, saturated to +-448, NaN kept);
+ * wm_advance moves codes; wm_attend attends over code * scale, i.e. exactly
+ * the dequantised prefix (the codes are widened to bf16 in the handle's
+ * scratch, 2 * C * heads * d * 2 bytes allocated here, and the scales enter
+ * in float32: K's with the softmax scale, V's with the output
+ * normalisation).  wm_write_attend is three launches (store, widen, attend).
+ * Calls on one E4M3 handle must be ordered on the device (one stream, or
+ * events between streams): they share its scratch.  wm_set_sink returns
+ * WM_ERR_UNSUPPORTED for this format.  Other arguments and errors as for
+ * wm_kvbuf_create; WM_ERR_INVALID_ARG for a missing or non-positive scale. */
+WM_API int wm_kvbuf_create_fp8(wm_kvbuf** out, int blocks, int heads, int d, int grid_h,
+                               int grid_w, int X, int Y, int W, const float* k_scale,
+                               const float* v_scale);
+
+/* WM_KV_BF16 or WM_KV_E4M3; WM_ERR_INVALID_ARG for a NULL handle. */
+WM_API int wm_kv_format(const wm_kvbuf* h);
+
 /* Free the buffers and the handle (synchronises the device first). */
 WM_API int wm_kvbuf_destroy(wm_kvbuf* h);
 
@@ -156,8 +184,9 @@ WM_API int64_t wm_capacity(const wm_kvbuf* h);            /* C */
 WM_API int64_t wm_current_frame(const wm_kvbuf* h);       /* last t passed to wm_advance, -1 before */
 WM_API int wm_raw_slot(const wm_kvbuf* h, int64_t t);     /* (t-1) mod (Y+1) for t >= 1; -1 for t < 1 */
 WM_API int wm_sum_slot(const wm_kvbuf* h, int64_t f);     /* (f-1) mod (W-Y) for f >= 1; -1 if none */
-/* Device pointers of block's K and V buffers, each [C, heads, d] bf16.  Owned
- * by the handle; valid until wm_kvbuf_destroy. */
+/* Device pointers of block's K and V buffers, each [C, heads, d] bf16 (E4M3
+ * codes, one byte each, for a WM_KV_E4M3 handle).  Owned by the handle; valid
+ * until wm_kvbuf_destroy. */
 WM_API int wm_kv_ptrs(const wm_kvbuf* h, int block, void** K, void** V);
 
 /* Synchronise the handle's device (the caller's current device is restored),
@@ -211,6 +240,27 @@ WM_API int64_t wm_layout_record_row(int grid_h, int grid_w, int X, int Y, int64_
  * fails; nothing is launched in those cases. */
 WM_API int wm_attend_dense(const void* Q, const void* K, const void* V, void* O, int64_t Lq, int64_t Lk,
                     int heads, int d, int* dev_status, wm_stream_t stream);
+
+/* Dense attention over caller-owned FP8 E4M3 keys and values: the
+ * full-resolution comparison point of wm_attend_dense for FP8 buffers.
+ *   O[i,h,:] = sum_j softmax_j(Q[i,h,:] . Kd[j,h,:] / sqrt(d)) Vd[j,h,:],  j < Lk,
+ * with Kd = code_value(K8) * k_scale[h] and Vd = code_value(V8) * v_scale[h]
+ * (the E4M3 reading of wm_kvbuf_create_fp8).  Q/O device [Lq, heads, d] bf16;
+ * K8/V8 device [Lk, heads, d] E4M3 codes; k_scale/v_scale device arrays of
+ * `heads` floats.  `scratch` is caller-owned device memory of at least
+ * wm_attend_dense_fp8_scratch_bytes(Lk, heads, d) bytes, 16-byte aligned,
+ * where the codes are widened to bf16; it must not be in use by another call
+ * until the stream has passed this one.  dev_status as for wm_attend_dense.
+ * Returns WM_ERR_INVALID_ARG for a NULL or misaligned pointer, an empty Q or
+ * K, more than 65535 heads or a scratch too small, WM_ERR_UNSUPPORTED for a
+ * head dimension other than 64 or 128, WM_ERR_CUDA if a launch fails. */
+WM_API int wm_attend_dense_fp8(const void* Q, const void* K8, const void* V8, const float* k_scale,
+                               const float* v_scale, void* O, int64_t Lq, int64_t Lk, int heads,
+                               int d, void* scratch, int64_t scratch_bytes, int* dev_status,
+                               wm_stream_t stream);
+/* Scratch bytes wm_attend_dense_fp8 needs: 2 * Lk * heads * d * 2 (-1 for
+ * arguments it rejects). */
+WM_API int64_t wm_attend_dense_fp8_scratch_bytes(int64_t Lk, int heads, int d);
 
 #ifdef __cplusplus
 }

@@ -24,10 +24,12 @@
 // Pipeline per warpgroup g and its tile j (= g, g+2, ...):
 //   wait S_full[g] -> load the S row into registers -> arrive S_free[g]
 //   (for d = 64, P has its own TMEM columns, so the MMA warp can already issue
-//   S_{j+2} into S_g while this tile's softmax runs) -> row max; the exponent
-//   reference m moves only when the max grows by more than 2^8 (the final
-//   division by l is exact either way) -> p = 2^(s*log2(e)/sqrt(d) - m) in
-//   registers (MUFU, optionally part on the FMA pipe) -> wait O_done[g] (P.V
+//   S_{j+2} into S_g while this tile's softmax runs) -> p = 2^(s*log2(e)/sqrt(d)
+//   - m) in registers (MUFU, part on the FMA pipe), where the exponent
+//   reference m is the row max of the warpgroup's first tile and stays put
+//   until a tile's exponentials would reach 2^16 (then that tile is redone
+//   with m raised to its max; the final division by l is exact either way), so
+//   no row max precedes the exponentials -> wait O_done[g] (P.V
 //   of tile j-2 finished: O_g is stable and P_g is free; waiting only now
 //   hides the MMA round trip behind the exponentials) -> rescale O_g if m
 //   moved -> P as bf16 into TMEM -> arrive P_full[g].
@@ -69,11 +71,6 @@ static_assert(256 * SOFTMAX_REGS + 128 * CONTROL_REGS <= NUM_THREADS * LAUNCH_RE
 // clocks); the drain after a timeout waits up to 0.2 s per operation,
 // whatever the limit.
 constexpr uint64_t DRAIN_LIMIT_CYCLES = 400000000ull;
-#ifndef WMKV_RESCALE_THRESHOLD
-#define WMKV_RESCALE_THRESHOLD 8.0f
-#endif
-// log2 units: O and l are rescaled only when the row max grows by more than 2^8
-constexpr float RESCALE_THRESHOLD = WMKV_RESCALE_THRESHOLD;
 
 template <int D>
 struct Cfg {
@@ -153,6 +150,94 @@ constexpr int poly_pairs_per_8() {
   return WMKV_POLY_PAIRS_PER_8 >= 0 ? WMKV_POLY_PAIRS_PER_8 : (D == 64 ? 3 : 0);
 }
 
+// Exponentials of a tile stay below 2^REF_HEADROOM (log2 units above the
+// reference): enough room that a stale reference rarely needs a redo, small
+// enough that p * v cannot overflow float32 for any |v| below 2^80.
+constexpr float REF_HEADROOM = 16.f;
+constexpr float REF_HEADROOM_EXP = 65536.f;  // 2^REF_HEADROOM
+
+// Largest of the 128 scores of a row: eight independent chains of
+// three-input max, then a tree.
+__device__ __forceinline__ float row_max(const float (&s)[128]) {
+  float mx[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) mx[c] = fmax3(s[c], s[c + 8], s[c + 16]);
+#pragma unroll
+  for (int c = 24; c < 120; c += 16)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mx[i] = fmax3(mx[i], s[c + i], s[c + 8 + i]);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[120 + i]);
+  return fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], fmax3(mx[5], mx[6], mx[7])));
+}
+
+// p = 2^(s * sl2 - m_ref) for the 128 scores of a row, packed to bf16 pairs,
+// and their sum.  POLY of every 8 column pairs take the FMA-pipe polynomial,
+// the rest MUFU.EX2.  Returns false if some exponential may have reached
+// 2^REF_HEADROOM: for MUFU lanes the sum shows it (it would be at least that
+// large, or not finite), for polynomial lanes the largest argument (the
+// polynomial's bit arithmetic is only valid below 2^128).  NaN scores make it
+// return false as well.
+template <int POLY>
+__device__ __forceinline__ bool exp_tile(const float (&s)[128], float sl2, float m_ref,
+                                         uint32_t (&pk)[64], float& sum) {
+  const f2 scale2 = f2_make(sl2, sl2);
+  const f2 negm2 = f2_make(-m_ref, -m_ref);
+  f2 acc0 = f2_make(0.f, 0.f), acc1 = acc0, acc2 = acc0, acc3 = acc0;
+  float xm[3] = {-INFINITY, -INFINITY, -INFINITY};  // largest polynomial-lane argument
+#pragma unroll
+  for (int pp = 0; pp < 64; ++pp) {
+    const f2 x = f2_fma(f2_make(s[2 * pp], s[2 * pp + 1]), scale2, negm2);
+    f2 e;
+    if (EXP_F16X2) {
+      e = exp2_f16x2(x);
+    } else if ((pp % 8) >= 8 - POLY) {
+      float x0, x1;
+      f2_split(x, x0, x1);
+      float& m = xm[(pp % 8) % 3];
+      m = fmax3(m, x0, x1);
+      e = exp2_poly2(x);
+    } else {
+      float x0, x1;
+      f2_split(x, x0, x1);
+      e = f2_make(ex2_approx(x0), ex2_approx(x1));
+    }
+    switch (pp % 4) {
+      case 0: acc0 = f2_add(acc0, e); break;
+      case 1: acc1 = f2_add(acc1, e); break;
+      case 2: acc2 = f2_add(acc2, e); break;
+      default: acc3 = f2_add(acc3, e); break;
+    }
+    float e0, e1;
+    f2_split(e, e0, e1);
+    pk[pp] = pack_bf16x2(e0, e1);
+  }
+  const f2 acc = f2_add(f2_add(acc0, acc1), f2_add(acc2, acc3));
+  float a_lo, a_hi;
+  f2_split(acc, a_lo, a_hi);
+  sum = a_lo + a_hi;
+  const bool poly_ok = POLY == 0 || fmax3(xm[0], xm[1], xm[2]) < REF_HEADROOM;
+  return sum < REF_HEADROOM_EXP && poly_ok;
+}
+
+// The softmax warps tell the MMA issuers that a warpgroup has read S or
+// written P with one arrival per warp: the TMEM loads / stores of the whole
+// warp have completed at tcgen05.wait (a warp-wide instruction), so after the
+// fence and a warp sync one lane can speak for the warp (4 arrivals per
+// warpgroup instead of 128).
+#ifndef WMKV_WARP_ARRIVE
+#define WMKV_WARP_ARRIVE 1
+#endif
+constexpr uint32_t SOFTMAX_ARRIVALS = WMKV_WARP_ARRIVE ? 4 : 128;
+__device__ __forceinline__ void softmax_arrive(uint32_t bar, int lane) {
+  if (WMKV_WARP_ARRIVE) {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar);
+  } else {
+    mbar_arrive(bar);
+  }
+}
+
 // Keys come in up to MAX_SEGS segments, each with its own K and V tensor
 // maps (row extent = the segment's length, so the rows past its end are
 // zero-filled).  Softmax attention does not depend on the order of the keys,
@@ -177,6 +262,9 @@ struct AttendParams {
   uint4* copy_dst[2];
   int64_t copy_n16;
   uint64_t wait_limit;  // SM cycles per bounded wait
+  // per-head factors of the stored keys and values (FP8 buffers), or null
+  const float* k_scale;
+  const float* v_scale;
 };
 
 // Segment and row of key tile j, and how many of its 128 rows are keys.
@@ -253,8 +341,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
     }
     for (int g = 0; g < 2; ++g) {
       mbar_init(bar(C::B_SFULL + g), 1);
-      mbar_init(bar(C::B_SFREE + g), 128);
-      mbar_init(bar(C::B_PFULL + g), 128);
+      mbar_init(bar(C::B_SFREE + g), SOFTMAX_ARRIVALS);
+      mbar_init(bar(C::B_PFULL + g), SOFTMAX_ARRIVALS);
       mbar_init(bar(C::B_ODONE + g), 1);
     }
     // the last P.V of each warpgroup commits once (one issuer per warpgroup
@@ -512,7 +600,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
     const uint32_t s_addr = tmem + lane_off + (wg ? C::S_COL1 : C::S_COL0);
     const uint32_t p_addr = tmem + lane_off + (wg ? C::P_COL1 : C::P_COL0);
     const uint32_t o_addr = tmem + lane_off + (wg ? C::O_COL1 : C::O_COL0);
-    const float sl2 = p.scale_log2;
+    const float sl2 = p.k_scale ? p.scale_log2 * p.k_scale[head] : p.scale_log2;
     float m_ref = -INFINITY;  // exponent reference (log2 units)
     float l_run = 0.f;
     bool ok = true;
@@ -530,7 +618,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
       tmem_wait_ld();
       if (C::P_SEP) {
         tc_fence_before();
-        mbar_arrive(bar(C::B_SFREE + wg));
+        softmax_arrive(bar(C::B_SFREE + wg), lane);
       }
       float s[128];
 #pragma unroll
@@ -543,60 +631,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
             if (c >= valid) s[c] = -INFINITY;
         }
       }
-      // row max: eight independent chains of three-input max, then a tree
-      float mx[8];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) mx[c] = fmax3(s[c], s[c + 8], s[c + 16]);
-#pragma unroll
-      for (int c = 24; c < 120; c += 16)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mx[i] = fmax3(mx[i], s[c + i], s[c + 8 + i]);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[120 + i]);
-      const float m_tile =
-          fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], fmax3(mx[5], mx[6], mx[7]))) * sl2;
+      // Exponent reference m_ref (log2 units).  The first tile of a warpgroup
+      // takes its row max; later tiles keep the reference of the earlier ones
+      // (the softmax does not depend on the reference: l and O carry the same
+      // factor and the final division removes it), so a tile's exponentials do
+      // not wait for its max.  A tile whose exponentials could reach
+      // 2^REF_HEADROOM -- some score far above the reference -- is caught
+      // afterwards by exp_tile and redone from the scores still in registers,
+      // with the reference raised to the tile's max (O and l rescaled).
       float alpha = 1.f;
       bool grow = false;
-      if (n == 0) {
-        m_ref = m_tile;
-      } else if (m_tile > m_ref + RESCALE_THRESHOLD) {
-        alpha = ex2_approx(m_ref - m_tile);
-        m_ref = m_tile;
-        grow = true;
-      }
-      // p = 2^(s * sl2 - m_ref), packed to bf16 pairs
-      const f2 scale2 = f2_make(sl2, sl2);
-      const f2 negm2 = f2_make(-m_ref, -m_ref);
-      f2 acc0 = f2_make(0.f, 0.f), acc1 = acc0, acc2 = acc0, acc3 = acc0;
+      if (n == 0) m_ref = row_max(s) * sl2;
       uint32_t pk[64];
-#pragma unroll
-      for (int pp = 0; pp < 64; ++pp) {
-        const f2 x = f2_fma(f2_make(s[2 * pp], s[2 * pp + 1]), scale2, negm2);
-        f2 e;
-        if (EXP_F16X2) {
-          e = exp2_f16x2(x);
-        } else if ((pp % 8) >= 8 - poly_pairs_per_8<D>()) {
-          e = exp2_poly2(x);
-        } else {
-          float x0, x1;
-          f2_split(x, x0, x1);
-          e = f2_make(ex2_approx(x0), ex2_approx(x1));
-        }
-        switch (pp % 4) {
-          case 0: acc0 = f2_add(acc0, e); break;
-          case 1: acc1 = f2_add(acc1, e); break;
-          case 2: acc2 = f2_add(acc2, e); break;
-          default: acc3 = f2_add(acc3, e); break;
-        }
-        float e0, e1;
-        f2_split(e, e0, e1);
-        pk[pp] = pack_bf16x2(e0, e1);
+      float tile_sum;
+      if (!exp_tile<poly_pairs_per_8<D>()>(s, sl2, m_ref, pk, tile_sum)) {
+        const float m_new = fmaxf(row_max(s) * sl2, m_ref);
+        alpha = ex2_approx(m_ref - m_new);
+        m_ref = m_new;
+        grow = true;
+        exp_tile<poly_pairs_per_8<D>()>(s, sl2, m_ref, pk, tile_sum);
       }
-      const f2 acc = f2_add(f2_add(acc0, acc1), f2_add(acc2, acc3));
-      float a_lo, a_hi;
-      f2_split(acc, a_lo, a_hi);
       // l is rescaled by alpha (1 unless the reference grew) before this tile's sum
-      l_run = l_run * alpha + (a_lo + a_hi);
+      l_run = l_run * alpha + tile_sum;
       if (n > 0) {
         // P.V of this warpgroup's previous tile has finished: O is stable, P is free
         ok = mbar_wait_bounded(bar(C::B_ODONE + wg), (n - 1) & 1, abort_flag, p.wait_limit);
@@ -627,7 +683,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
       tmem_st32_at<32>(p_addr + 32, pk);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(C::B_PFULL + wg));
+      softmax_arrive(bar(C::B_PFULL + wg), lane);
     }
     // all P.V products must have landed before O is read
     if (ok) {
@@ -644,7 +700,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
       const float mf = fmaxf(m0, m1);
       const float a0 = ex2_approx(m0 - mf);
       const float a1 = ex2_approx(m1 - mf);
-      const float inv = 1.f / (l0 * a0 + l1 * a1);
+      const float inv = (p.v_scale ? p.v_scale[head] : 1.f) / (l0 * a0 + l1 * a1);
       const float c0 = a0 * inv, c1 = a1 * inv;
       const bool has1 = nkv > 1;
       const int64_t qrow = int64_t(q_tile) * BM + row;
@@ -751,7 +807,8 @@ bool attend_copies_in_kernel(int d) { return Cfg<64>::COPY_IN_KERNEL && d == 64;
 
 cudaError_t launch_attend(const void* q, void* o, int64_t lq, const KVSegment* segs, int nseg,
                           int heads, int d, int* status, const RecordCopy* copy,
-                          unsigned long long wait_limit, cudaStream_t stream) {
+                          unsigned long long wait_limit, const float* k_scale,
+                          const float* v_scale, cudaStream_t stream) {
   if (nseg < 1 || nseg > MAX_SEGS) return cudaErrorInvalidValue;
   AttendParams prm = {};
   if (!encode_rows_map(&prm.tm_q, q, lq, heads, d)) return cudaErrorInvalidValue;
@@ -772,6 +829,8 @@ cudaError_t launch_attend(const void* q, void* o, int64_t lq, const KVSegment* s
   prm.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
   prm.status = status;
   prm.wait_limit = wait_limit;
+  prm.k_scale = k_scale;
+  prm.v_scale = v_scale;
   if (copy && copy->n16 > 0) {
     if (!attend_copies_in_kernel(d)) return cudaErrorInvalidValue;
     prm.copy_src[0] = static_cast<const uint4*>(copy->k_src);

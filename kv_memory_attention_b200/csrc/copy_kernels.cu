@@ -113,8 +113,10 @@ __global__ void __launch_bounds__(COPY_THREADS) rotate_z0_kernel(uint8_t* base, 
   *v = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+}  // namespace
+
 // SM count of the current device (queried once per device, thread-safe).
-int sm_count() {
+int device_sm_count() {
   constexpr int MAX_DEVICES = 64;
   static std::once_flag once[MAX_DEVICES];
   static int count[MAX_DEVICES];
@@ -129,12 +131,14 @@ int sm_count() {
   return count[dev];
 }
 
+namespace {
+
 unsigned grid_x_for(int64_t n16, int parallel_arrays) {
   // enough CTAs for every vector to be touched once with UNROLL in flight,
   // capped at a few waves of the SM count across all arrays
   const int64_t per_cta = int64_t(COPY_THREADS) * UNROLL;
   int64_t want = (n16 + per_cta - 1) / per_cta;
-  const int64_t cap = (int64_t(sm_count()) * 8 + parallel_arrays - 1) / parallel_arrays;
+  const int64_t cap = (int64_t(device_sm_count()) * 8 + parallel_arrays - 1) / parallel_arrays;
   if (want > cap) want = cap;
   if (want < 1) want = 1;
   return static_cast<unsigned>(want);

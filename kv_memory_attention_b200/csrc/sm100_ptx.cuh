@@ -343,7 +343,8 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// 2^x on the FMA pipe, for x <= 0 (softmax exponents).  Cody-Waite style
+// 2^x on the FMA pipe for x in [-125, 127] (softmax exponents: the attention
+// keeps them below 2^16 and checks that it did).  Cody-Waite style
 // reduction x = j + f with j = round(x), f in [-1/2, 1/2] (W. J. Cody and
 // W. Waite, "Software Manual for the Elementary Functions", 1980): j is read
 // from the low mantissa bits of x + 1.5*2^23, 2^f is a minimax polynomial
@@ -351,8 +352,10 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // error over [-1/2, 1/2]: cubic 7.5e-5 = 2^-13.7, quadratic 1.7e-3 = 2^-9.2,
 // the latter about the size of the bf16 rounding P gets anyway), and 2^j is
 // added into the exponent field.  x is clamped at -125 so the result stays a
-// normal float; anything below 2^-125 is negligible next to the row maximum
-// of a softmax (which is 1).  Two lanes per call (f32x2).
+// normal float; anything below 2^-125 is negligible next to the largest term
+// of a softmax row (at least 1).  Above 127 the exponent field overflows and
+// the result is meaningless, which the caller must rule out.  Two lanes per
+// call (f32x2).
 #ifndef WMKV_POLY_DEGREE
 #define WMKV_POLY_DEGREE 2
 #endif

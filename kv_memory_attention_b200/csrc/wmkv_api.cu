@@ -26,11 +26,16 @@ struct wm_kvbuf {
   int device = 0;
   int blocks = 0, heads = 0, d = 0, grid_h = 0, grid_w = 0, X = 0, Y = 0, W = 0;
   int64_t HW = 0, R = 0, C = 0;
-  int64_t row_bytes = 0;     // heads * d * 2
+  int kv_format = WM_KV_BF16;
+  int64_t row_bytes = 0;     // heads * d * (2 for bf16, 1 for E4M3 codes)
   int64_t tensor_bytes = 0;  // C * row_bytes (one K or V buffer)
   int64_t block_bytes = 0;   // 2 * tensor_bytes
   uint8_t* buf = nullptr;
   int* status = nullptr;     // device error word
+  // E4M3 buffers: per (block, head) scales on the device (K for all blocks,
+  // then V), and the bf16 widening of one block's filled prefix (K, then V)
+  float* scales = nullptr;
+  uint8_t* widened = nullptr;
   int64_t t = -1;            // current frame
   std::vector<int64_t> written;  // per block: frame of the latest write_record
   // streaming sink (start image keys follow the window)
@@ -93,17 +98,25 @@ int64_t record_row(int64_t hw, int64_t X, int64_t Y, int64_t t) {
 
 extern "C" {
 
-int wm_kvbuf_create(wm_kvbuf** out, int blocks, int heads, int d, int grid_h, int grid_w, int X,
-                    int Y, int W) {
+static int kvbuf_create(wm_kvbuf** out, int blocks, int heads, int d, int grid_h, int grid_w, int X,
+                        int Y, int W, int kv_format, const float* k_scale, const float* v_scale) {
   if (!out) return WM_ERR_INVALID_ARG;
   *out = nullptr;
   if (blocks < 1 || heads < 1 || heads > 65535 || grid_h < 1 || grid_w < 1 || X < 1 || Y < 0 ||
       W < Y)
     return WM_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return WM_ERR_UNSUPPORTED;
+  const int elem_bytes = kv_format == WM_KV_E4M3 ? 1 : 2;
+  if (kv_format == WM_KV_E4M3) {
+    if (!k_scale || !v_scale) return WM_ERR_INVALID_ARG;
+    for (int64_t i = 0; i < int64_t(blocks) * heads; ++i)
+      if (!(k_scale[i] > 0.f) || !(v_scale[i] > 0.f) || !std::isfinite(k_scale[i]) ||
+          !std::isfinite(v_scale[i]))
+        return WM_ERR_INVALID_ARG;
+  }
   const int64_t hw = int64_t(grid_h) * grid_w;
   const int64_t C = capacity(hw, X, Y, W);
-  const int64_t row_bytes = int64_t(heads) * d * 2;
+  const int64_t row_bytes = int64_t(heads) * d * elem_bytes;
   // rows are addressed with 32-bit TMA coordinates
   if (C >= (int64_t(1) << 31) || hw + X >= (int64_t(1) << 31)) return WM_ERR_INVALID_ARG;
   const int64_t tensor_bytes = C * row_bytes;
@@ -123,39 +136,56 @@ int wm_kvbuf_create(wm_kvbuf** out, int blocks, int heads, int d, int grid_h, in
   h->HW = hw;
   h->R = hw + X;
   h->C = C;
+  h->kv_format = kv_format;
   h->row_bytes = row_bytes;
   h->tensor_bytes = tensor_bytes;
   h->block_bytes = 2 * tensor_bytes;
   h->written.assign(blocks, -1);
 
-  cudaError_t e = cudaGetDevice(&h->device);
-  if (e != cudaSuccess) {
-    delete h;
-    return cuda_fail(e);
-  }
-  const size_t total = size_t(h->block_bytes) * size_t(blocks);
-  e = cudaMalloc(&h->buf, total);
-  if (e != cudaSuccess) {
+  auto fail = [h](cudaError_t e) -> int {
+    cudaFree(h->buf);
+    cudaFree(h->status);
+    cudaFree(h->scales);
+    cudaFree(h->widened);
     delete h;
     if (e == cudaErrorMemoryAllocation) {
       cudaGetLastError();
       return WM_ERR_OOM;
     }
     return cuda_fail(e);
+  };
+  cudaError_t e = cudaGetDevice(&h->device);
+  if (e != cudaSuccess) return fail(e);
+  const size_t total = size_t(h->block_bytes) * size_t(blocks);
+  e = cudaMalloc(&h->buf, total);
+  if (e == cudaSuccess) e = cudaMalloc(&h->status, sizeof(int));
+  if (e == cudaSuccess && kv_format == WM_KV_E4M3) {
+    const size_t ns = size_t(blocks) * heads;
+    e = cudaMalloc(&h->scales, 2 * ns * sizeof(float));
+    if (e == cudaSuccess) e = cudaMemcpy(h->scales, k_scale, ns * sizeof(float), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess)
+      e = cudaMemcpy(h->scales + ns, v_scale, ns * sizeof(float), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMalloc(&h->widened, size_t(2) * C * heads * d * 2);
   }
-  e = cudaMalloc(&h->status, sizeof(int));
   if (e == cudaSuccess) e = cudaMemset(h->buf, 0, total);
   if (e == cudaSuccess) e = cudaMemset(h->status, 0, sizeof(int));
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
-  if (e != cudaSuccess) {
-    cudaFree(h->buf);
-    if (h->status) cudaFree(h->status);
-    delete h;
-    return cuda_fail(e);
-  }
+  if (e != cudaSuccess) return fail(e);
   *out = h;
   return WM_OK;
 }
+
+int wm_kvbuf_create(wm_kvbuf** out, int blocks, int heads, int d, int grid_h, int grid_w, int X,
+                    int Y, int W) {
+  return kvbuf_create(out, blocks, heads, d, grid_h, grid_w, X, Y, W, WM_KV_BF16, nullptr, nullptr);
+}
+
+int wm_kvbuf_create_fp8(wm_kvbuf** out, int blocks, int heads, int d, int grid_h, int grid_w,
+                        int X, int Y, int W, const float* k_scale, const float* v_scale) {
+  return kvbuf_create(out, blocks, heads, d, grid_h, grid_w, X, Y, W, WM_KV_E4M3, k_scale, v_scale);
+}
+
+int wm_kv_format(const wm_kvbuf* h) { return h ? h->kv_format : WM_ERR_INVALID_ARG; }
 
 int wm_kvbuf_destroy(wm_kvbuf* h) {
   if (!h) return WM_ERR_INVALID_ARG;
@@ -165,6 +195,8 @@ int wm_kvbuf_destroy(wm_kvbuf* h) {
   cudaError_t e = cudaDeviceSynchronize();
   cudaFree(h->buf);
   cudaFree(h->status);
+  cudaFree(h->scales);
+  cudaFree(h->widened);
   cudaSetDevice(dev);
   delete h;
   return e == cudaSuccess ? WM_OK : cuda_fail(e);
@@ -211,6 +243,7 @@ int wm_advance(wm_kvbuf* h, int64_t t, wm_stream_t stream) {
 int wm_set_sink(wm_kvbuf* h, const float* theta, int n_pairs, int gap_trigger, int gap_target) {
   if (!h || !theta || n_pairs != h->d / 2 || gap_target < 0 || gap_trigger <= gap_target)
     return WM_ERR_INVALID_ARG;
+  if (h->kv_format != WM_KV_BF16) return WM_ERR_UNSUPPORTED;
   if (h->t >= 0) return WM_ERR_STATE;
   h->theta.assign(theta, theta + n_pairs);
   h->gap_trigger = gap_trigger;
@@ -233,16 +266,50 @@ int wm_sink_cos_sin(const wm_kvbuf* h, int64_t shift, float* c, float* s) {
   return WM_OK;
 }
 
+// Scales of block b (device): K's heads, V's heads.
+static const float* block_k_scale(const wm_kvbuf* h, int b) { return h->scales + int64_t(b) * h->heads; }
+static const float* block_v_scale(const wm_kvbuf* h, int b) {
+  return h->scales + (int64_t(h->blocks) + b) * h->heads;
+}
+
+// Store a bf16 record [R, heads, d] into rows starting at row0 of block b.
+static cudaError_t store_record(wm_kvbuf* h, int block, int64_t row0, const void* K, const void* V,
+                                cudaStream_t s) {
+  uint8_t* kdst = h->buf + int64_t(block) * h->block_bytes + row0 * h->row_bytes;
+  uint8_t* vdst = kdst + h->tensor_bytes;
+  if (h->kv_format == WM_KV_E4M3)
+    return wmkv::launch_quantize_pair(K, V, kdst, vdst, h->R * h->heads * h->d, h->heads, h->d,
+                                      block_k_scale(h, block), block_v_scale(h, block), s);
+  return wmkv::launch_copy_pair(K, V, kdst, vdst, h->R * h->row_bytes / 16, s);
+}
+
+// Attention of Q over buffer[0:end] of block b; an E4M3 buffer is first
+// widened into the handle's bf16 scratch and attended with its scales.
+static cudaError_t attend_prefix(wm_kvbuf* h, int block, const void* Q, void* O, cudaStream_t s) {
+  const int64_t end = end_at(h->HW, h->X, h->Y, h->W, h->t);
+  const uint8_t* kbuf = h->buf + int64_t(block) * h->block_bytes;
+  const uint8_t* vbuf = kbuf + h->tensor_bytes;
+  if (h->kv_format == WM_KV_E4M3) {
+    uint8_t* wk = h->widened;
+    uint8_t* wv = h->widened + h->C * h->heads * h->d * 2;
+    cudaError_t e = wmkv::launch_widen_pair(kbuf, vbuf, wk, wv, end * h->heads * h->d, s);
+    if (e != cudaSuccess) return e;
+    const wmkv::KVSegment seg = {wk, wv, end};
+    return wmkv::launch_attend(Q, O, h->R, &seg, 1, h->heads, h->d, h->status, nullptr, h->wait_limit,
+                               block_k_scale(h, block), block_v_scale(h, block), s);
+  }
+  const wmkv::KVSegment seg = {kbuf, vbuf, end};
+  return wmkv::launch_attend(Q, O, h->R, &seg, 1, h->heads, h->d, h->status, nullptr, h->wait_limit,
+                             nullptr, nullptr, s);
+}
+
 int wm_write_record(wm_kvbuf* h, int block, int64_t t, const void* K, const void* V,
                     wm_stream_t stream) {
   if (!h || block < 0 || block >= h->blocks || !aligned16(K) || !aligned16(V))
     return WM_ERR_INVALID_ARG;
   if (h->t < 0 || t != h->t || !on_handle_device(h)) return WM_ERR_STATE;
   const int64_t row0 = record_row(h->HW, h->X, h->Y, t);
-  uint8_t* kdst = h->buf + int64_t(block) * h->block_bytes + row0 * h->row_bytes;
-  uint8_t* vdst = kdst + h->tensor_bytes;
-  const int64_t n16 = h->R * h->row_bytes / 16;
-  cudaError_t e = wmkv::launch_copy_pair(K, V, kdst, vdst, n16, reinterpret_cast<cudaStream_t>(stream));
+  cudaError_t e = store_record(h, block, row0, K, V, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
   h->written[block] = t;
   return WM_OK;
@@ -252,12 +319,7 @@ int wm_attend(wm_kvbuf* h, int block, const void* Q, void* O, wm_stream_t stream
   if (!h || block < 0 || block >= h->blocks || !aligned16(Q) || !aligned16(O))
     return WM_ERR_INVALID_ARG;
   if (h->t < 0 || h->written[block] != h->t || !on_handle_device(h)) return WM_ERR_STATE;
-  const int64_t end = end_at(h->HW, h->X, h->Y, h->W, h->t);
-  const uint8_t* kbuf = h->buf + int64_t(block) * h->block_bytes;
-  const uint8_t* vbuf = kbuf + h->tensor_bytes;
-  const wmkv::KVSegment seg = {kbuf, vbuf, end};
-  cudaError_t e = wmkv::launch_attend(Q, O, h->R, &seg, 1, h->heads, h->d, h->status, nullptr,
-                                      h->wait_limit, reinterpret_cast<cudaStream_t>(stream));
+  cudaError_t e = attend_prefix(h, block, Q, O, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
   return WM_OK;
 }
@@ -283,7 +345,12 @@ int wm_write_attend(wm_kvbuf* h, int block, int64_t t, const void* Q, const void
   const int64_t n16 = h->R * h->row_bytes / 16;
   const int64_t end = end_at(h->HW, h->X, h->Y, h->W, t);
   cudaError_t e;
-  if (wmkv::attend_copies_in_kernel(h->d)) {
+  if (h->kv_format == WM_KV_E4M3) {
+    // the attention must see the stored (quantised) record: store, then attend
+    h->written[block] = -1;
+    e = store_record(h, block, row0, K, V, s);
+    if (e == cudaSuccess) e = attend_prefix(h, block, Q, O, s);
+  } else if (wmkv::attend_copies_in_kernel(h->d)) {
     // keys: buffer rows before the slot, buffer rows after it, and the record
     // itself from the caller (the slot is being written by the same launch)
     wmkv::KVSegment segs[3];
@@ -295,13 +362,13 @@ int wm_write_attend(wm_kvbuf* h, int block, int64_t t, const void* Q, const void
     segs[nseg++] = {K, V, h->R};
     const wmkv::RecordCopy cp = {K, V, kslot, vslot, n16};
     e = wmkv::launch_attend(Q, O, h->R, segs, nseg, h->heads, h->d, h->status, &cp, h->wait_limit,
-                            s);
+                            nullptr, nullptr, s);
   } else {
     e = wmkv::launch_copy_pair(K, V, kslot, vslot, n16, s);
     const wmkv::KVSegment seg = {kbuf, vbuf, end};
     if (e == cudaSuccess)
       e = wmkv::launch_attend(Q, O, h->R, &seg, 1, h->heads, h->d, h->status, nullptr,
-                              h->wait_limit, s);
+                              h->wait_limit, nullptr, nullptr, s);
   }
   if (e != cudaSuccess) return cuda_fail(e);
   h->written[block] = t;
@@ -382,8 +449,34 @@ int wm_attend_dense(const void* Q, const void* K, const void* V, void* O, int64_
   if ((Lq + 127) / 128 > 0x7FFFFFFF || heads > 65535) return WM_ERR_INVALID_ARG;
   const wmkv::KVSegment seg = {K, V, Lk};
   cudaError_t e = wmkv::launch_attend(Q, O, Lq, &seg, 1, heads, d, dev_status, nullptr,
-                                      wmkv::DEFAULT_WAIT_LIMIT_CYCLES,
+                                      wmkv::DEFAULT_WAIT_LIMIT_CYCLES, nullptr, nullptr,
                                       reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return WM_OK;
+}
+
+int64_t wm_attend_dense_fp8_scratch_bytes(int64_t Lk, int heads, int d) {
+  if (Lk < 1 || heads < 1 || (d != 64 && d != 128)) return -1;
+  return 2 * Lk * heads * d * 2;
+}
+
+int wm_attend_dense_fp8(const void* Q, const void* K8, const void* V8, const float* k_scale,
+                        const float* v_scale, void* O, int64_t Lq, int64_t Lk, int heads, int d,
+                        void* scratch, int64_t scratch_bytes, int* dev_status, wm_stream_t stream) {
+  if (!aligned16(Q) || !aligned16(K8) || !aligned16(V8) || !aligned16(O) || !aligned16(scratch) ||
+      !k_scale || !v_scale || Lq < 1 || Lk < 1 || heads < 1 || heads > 65535 ||
+      Lq >= (int64_t(1) << 31) || Lk >= (int64_t(1) << 31))
+    return WM_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return WM_ERR_UNSUPPORTED;
+  if (scratch_bytes < wm_attend_dense_fp8_scratch_bytes(Lk, heads, d)) return WM_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* wk = static_cast<uint8_t*>(scratch);
+  uint8_t* wv = wk + Lk * heads * d * 2;
+  cudaError_t e = wmkv::launch_widen_pair(K8, V8, wk, wv, Lk * heads * d, s);
+  const wmkv::KVSegment seg = {wk, wv, Lk};
+  if (e == cudaSuccess)
+    e = wmkv::launch_attend(Q, O, Lq, &seg, 1, heads, d, dev_status, nullptr,
+                            wmkv::DEFAULT_WAIT_LIMIT_CYCLES, k_scale, v_scale, s);
   if (e != cudaSuccess) return cuda_fail(e);
   return WM_OK;
 }

@@ -60,10 +60,28 @@ struct RecordCopy {
 // the 1.965 GHz maximum clock).
 constexpr unsigned long long DEFAULT_WAIT_LIMIT_CYCLES = 4000000000ull;
 
+// k_scale / v_scale (device, one float per head, may be null): the keys and
+// values are the stored numbers times their head's scale (FP8 buffers).
 cudaError_t launch_attend(const void* q, void* o, int64_t lq, const KVSegment* segs, int nseg,
                           int heads, int d, int* status, const RecordCopy* copy,
-                          unsigned long long wait_limit, cudaStream_t stream);
+                          unsigned long long wait_limit, const float* k_scale,
+                          const float* v_scale, cudaStream_t stream);
 bool attend_copies_in_kernel(int d);
+
+// SM count of the current device (queried once per device).
+int device_sm_count();
+
+// FP8 (E4M3) buffers.  Quantise `elems` bf16 values of K and of V ([rows,
+// heads, d], elems a multiple of 8) into codes with one scale per head
+// (device arrays of `heads` floats): code = E4M3(x / scale), round to nearest
+// even, saturate to +-448.
+cudaError_t launch_quantize_pair(const void* k_src, const void* v_src, void* k_dst, void* v_dst,
+                                 int64_t elems, int heads, int d, const float* k_scale,
+                                 const float* v_scale, cudaStream_t stream);
+// Widen `elems` E4M3 codes of K and of V (elems a multiple of 16) to the
+// bfloat16 values they hold (exact).
+cudaError_t launch_widen_pair(const void* k_codes, const void* v_codes, void* k_out, void* v_out,
+                              int64_t elems, cudaStream_t stream);
 
 // Copy `n16` 16-byte chunks of a and b (two independent arrays) in one launch.
 cudaError_t launch_copy_pair(const void* a_src, const void* b_src, void* a_dst, void* b_dst,

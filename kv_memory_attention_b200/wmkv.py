@@ -27,6 +27,10 @@ _c_int, _c_i64, _vp = ctypes.c_int, ctypes.c_int64, ctypes.c_void_p
 SIGNATURES = {
     "wm_kvbuf_create": (_c_int, [ctypes.POINTER(_vp), _c_int, _c_int, _c_int, _c_int, _c_int,
                                  _c_int, _c_int, _c_int]),
+    "wm_kvbuf_create_fp8": (_c_int, [ctypes.POINTER(_vp), _c_int, _c_int, _c_int, _c_int, _c_int,
+                                     _c_int, _c_int, _c_int, ctypes.POINTER(ctypes.c_float),
+                                     ctypes.POINTER(ctypes.c_float)]),
+    "wm_kv_format": (_c_int, [_vp]),
     "wm_kvbuf_destroy": (_c_int, [_vp]),
     "wm_advance": (_c_int, [_vp, _c_i64, _vp]),
     "wm_write_record": (_c_int, [_vp, _c_int, _c_i64, _vp, _vp, _vp]),
@@ -52,7 +56,13 @@ SIGNATURES = {
     "wm_layout_sum_slot": (_c_int, [_c_int, _c_int, _c_i64]),
     "wm_layout_record_row": (_c_i64, [_c_int, _c_int, _c_int, _c_int, _c_i64]),
     "wm_attend_dense": (_c_int, [_vp, _vp, _vp, _vp, _c_i64, _c_i64, _c_int, _c_int, _vp, _vp]),
+    "wm_attend_dense_fp8": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _c_i64, _c_i64, _c_int, _c_int,
+                                     _vp, _c_i64, _vp, _vp]),
+    "wm_attend_dense_fp8_scratch_bytes": (_c_i64, [_c_i64, _c_int, _c_int]),
 }
+
+WM_KV_BF16 = 0
+WM_KV_E4M3 = 1
 
 
 def _load():
@@ -111,6 +121,24 @@ def wm_kvbuf_create(blocks: int, heads: int, d: int, grid_h: int, grid_w: int, X
     _check(LIB.wm_kvbuf_create(ctypes.byref(h), blocks, heads, d, grid_h, grid_w, X, Y, W),
            "wm_kvbuf_create")
     return h.value
+
+
+def wm_kvbuf_create_fp8(blocks: int, heads: int, d: int, grid_h: int, grid_w: int, X: int, Y: int,
+                        W: int, k_scale, v_scale) -> int:
+    """k_scale / v_scale: blocks * heads floats each (block-major)."""
+    n = blocks * heads
+    if len(k_scale) != n or len(v_scale) != n:
+        raise ValueError(f"expected {n} scales per tensor")
+    ks = (ctypes.c_float * n)(*[float(x) for x in k_scale])
+    vs = (ctypes.c_float * n)(*[float(x) for x in v_scale])
+    h = _vp()
+    _check(LIB.wm_kvbuf_create_fp8(ctypes.byref(h), blocks, heads, d, grid_h, grid_w, X, Y, W, ks, vs),
+           "wm_kvbuf_create_fp8")
+    return h.value
+
+
+def wm_kv_format(h: int) -> int:
+    return LIB.wm_kv_format(h)
 
 
 def wm_kvbuf_destroy(h: int) -> None:
@@ -197,6 +225,17 @@ def wm_attend_dense(Q, K, V, O, Lq: int, Lk: int, heads: int, d: int, dev_status
                                _ptr(dev_status), _stream(stream)), "wm_attend_dense")
 
 
+def wm_attend_dense_fp8_scratch_bytes(Lk: int, heads: int, d: int) -> int:
+    return LIB.wm_attend_dense_fp8_scratch_bytes(Lk, heads, d)
+
+
+def wm_attend_dense_fp8(Q, K8, V8, k_scale, v_scale, O, Lq: int, Lk: int, heads: int, d: int,
+                        scratch, scratch_bytes: int, dev_status=None, stream=None) -> None:
+    _check(LIB.wm_attend_dense_fp8(_ptr(Q), _ptr(K8), _ptr(V8), _ptr(k_scale), _ptr(v_scale), _ptr(O),
+                                   Lq, Lk, heads, d, _ptr(scratch), scratch_bytes, _ptr(dev_status),
+                                   _stream(stream)), "wm_attend_dense_fp8")
+
+
 def wm_layout_capacity(grid_h, grid_w, X, Y, W) -> int:
     return LIB.wm_layout_capacity(grid_h, grid_w, X, Y, W)
 
@@ -227,12 +266,21 @@ class KVMemory:
     calls that wrote them).
     """
 
-    def __init__(self, blocks, heads, d, grid_h, grid_w, X, Y, W):
+    def __init__(self, blocks, heads, d, grid_h, grid_w, X, Y, W, kv_format="bf16",
+                 k_scale=None, v_scale=None):
         self.blocks, self.heads, self.d = blocks, heads, d
         self.grid_h, self.grid_w, self.X, self.Y, self.W = grid_h, grid_w, X, Y, W
         self.HW = grid_h * grid_w
         self.R = self.HW + X
-        self.h = wm_kvbuf_create(blocks, heads, d, grid_h, grid_w, X, Y, W)
+        self.kv_format = kv_format
+        self.h = None
+        if kv_format == "bf16":
+            self.h = wm_kvbuf_create(blocks, heads, d, grid_h, grid_w, X, Y, W)
+        elif kv_format == "e4m3":
+            self.h = wm_kvbuf_create_fp8(blocks, heads, d, grid_h, grid_w, X, Y, W,
+                                         list(k_scale), list(v_scale))
+        else:
+            raise ValueError(kv_format)
         self.C = wm_capacity(self.h)
 
     def close(self):
@@ -274,22 +322,25 @@ class KVMemory:
         wm_set_wait_limit(self.h, cycles)
 
     def kv_views(self, block):
+        """Torch views of the block's buffers: bf16, or uint8 E4M3 codes."""
         import torch
         kp, vp = wm_kv_ptrs(self.h, block)
         n = self.C * self.heads * self.d
-        return (_device_view(kp, n, torch.bfloat16).view(self.C, self.heads, self.d),
-                _device_view(vp, n, torch.bfloat16).view(self.C, self.heads, self.d))
+        dt = torch.uint8 if self.kv_format == "e4m3" else torch.bfloat16
+        return (_device_view(kp, n, dt).view(self.C, self.heads, self.d),
+                _device_view(vp, n, dt).view(self.C, self.heads, self.d))
 
 
 def _device_view(ptr: int, numel: int, dtype):
     """A torch tensor aliasing library-owned device memory (no copy, no ownership)."""
     import torch
+    one_byte = dtype == torch.uint8
 
     class _Holder:
-        def __init__(self, p, nbytes):
+        def __init__(self, p, n):
             self.__cuda_array_interface__ = {
-                "shape": (nbytes // 2,), "typestr": "<i2", "data": (p, False), "version": 3,
-                "strides": None}
+                "shape": (n,), "typestr": "|u1" if one_byte else "<i2", "data": (p, False),
+                "version": 3, "strides": None}
 
-    t = torch.as_tensor(_Holder(ptr, numel * 2), device="cuda")
-    return t.view(dtype)
+    t = torch.as_tensor(_Holder(ptr, numel), device="cuda")
+    return t if one_byte else t.view(dtype)

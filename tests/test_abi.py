@@ -100,6 +100,30 @@ def test_null_handle_and_pointer_errors(wm):
     assert lib.wm_attend_dense(16, 16, 16, 16, 1, 1, 1, 80, None, None) == wm.WM_ERR_UNSUPPORTED
 
 
+def test_fp8_argument_checks(wm):
+    lib = wm.LIB
+    h = ctypes.c_void_p()
+    ones = (ctypes.c_float * 4)(1.0, 1.0, 1.0, 1.0)
+    bad = (ctypes.c_float * 4)(1.0, 0.0, 1.0, 1.0)
+    nan = (ctypes.c_float * 4)(1.0, float("nan"), 1.0, 1.0)
+    args = (2, 2, 64, 4, 6, 4, 2, 6)
+    assert lib.wm_kvbuf_create_fp8(ctypes.byref(h), *args, None, ones) == wm.WM_ERR_INVALID_ARG
+    assert lib.wm_kvbuf_create_fp8(ctypes.byref(h), *args, ones, bad) == wm.WM_ERR_INVALID_ARG
+    assert lib.wm_kvbuf_create_fp8(ctypes.byref(h), *args, nan, ones) == wm.WM_ERR_INVALID_ARG
+    assert lib.wm_kvbuf_create_fp8(ctypes.byref(h), 2, 2, 96, 4, 6, 4, 2, 6, ones, ones) == \
+        wm.WM_ERR_UNSUPPORTED
+    assert lib.wm_kv_format(None) == wm.WM_ERR_INVALID_ARG
+    assert wm.wm_attend_dense_fp8_scratch_bytes(1000, 3, 64) == 2 * 1000 * 3 * 64 * 2
+    assert wm.wm_attend_dense_fp8_scratch_bytes(0, 3, 64) == -1
+    assert wm.wm_attend_dense_fp8_scratch_bytes(10, 3, 80) == -1
+    f = lib.wm_attend_dense_fp8
+    assert f(16, 16, 16, None, 16, 16, 1, 1, 1, 64, 16, 256, None, None) == wm.WM_ERR_INVALID_ARG
+    assert f(16, 16, 24, 16, 16, 16, 1, 1, 1, 64, 16, 256, None, None) == wm.WM_ERR_INVALID_ARG
+    assert f(16, 16, 16, 16, 16, 16, 1, 1, 1, 64, 16, 255, None, None) == wm.WM_ERR_INVALID_ARG
+    assert f(16, 16, 16, 16, 16, 16, 1, 0, 1, 64, 16, 256, None, None) == wm.WM_ERR_INVALID_ARG
+    assert f(16, 16, 16, 16, 16, 16, 1, 1, 1, 96, 16, 1 << 20, None, None) == wm.WM_ERR_UNSUPPORTED
+
+
 def test_strerror_covers_codes(wm):
     for c in range(0, -7, -1):
         assert wm.wm_strerror(c) and wm.wm_strerror(c) != "unknown error"

@@ -42,12 +42,12 @@ def test_copy_byte_counts():
 
 NCU_CSV = '''==PROF== Connected to process 123
 "ID","Process ID","Process Name","Host Name","Kernel Name","Context","Stream","Block Size","Grid Size","Device","CC","Section Name","Metric Name","Metric Unit","Metric Value"
-"0","123","python3","127.0.0.1","void wmkv::(anonymous namespace)::evict_kernel(unsigned char *, long, long, long, long, long)","1","7","(256, 1, 1)","(12, 56, 1)","0","10.0","Command line profiler metrics","gpu__time_duration.sum","usecond","6.00"
+"0","123","python3","127.0.0.1","void wmkv::(anonymous namespace)::evict_kernel(unsigned char *, long, long, long, long, long)","1","7","(256, 1, 1)","(12, 56, 1)","0","10.0","Command line profiler metrics","gpu__time_duration.sum","us","6.00"
 "1","123","python3","127.0.0.1","void wmkv::(anonymous namespace)::attend_kernel<64>(wmkv::(anonymous namespace)::AttendParams)","1","7","(384, 1, 1)","(9, 16, 1)","0","10.0","Command line profiler metrics","gpu__time_duration.sum","usecond","50.00"
 "1","123","python3","127.0.0.1","void wmkv::(anonymous namespace)::attend_kernel<64>(wmkv::(anonymous namespace)::AttendParams)","1","7","(384, 1, 1)","(9, 16, 1)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","Mbyte","29.05"
 "1","123","python3","127.0.0.1","void wmkv::(anonymous namespace)::attend_kernel<64>(wmkv::(anonymous namespace)::AttendParams)","1","7","(384, 1, 1)","(9, 16, 1)","0","10.0","Command line profiler metrics","dram__bytes_write.sum","Kbyte","8.00"
-"2","123","python3","127.0.0.1","void wmkv::(anonymous namespace)::attend_kernel<64>(wmkv::(anonymous namespace)::AttendParams)","1","7","(384, 1, 1)","(9, 16, 1)","0","10.0","Command line profiler metrics","gpu__time_duration.sum","nsecond","54,000"
-"2","123","python3","127.0.0.1","void wmkv::(anonymous namespace)::attend_kernel<64>(wmkv::(anonymous namespace)::AttendParams)","1","7","(384, 1, 1)","(9, 16, 1)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","byte","29,050,000"
+"2","123","python3","127.0.0.1","void wmkv::(anonymous namespace)::attend_kernel<64>(wmkv::(anonymous namespace)::AttendParams)","1","7","(384, 1, 1)","(9, 16, 1)","0","10.0","Command line profiler metrics","gpu__time_duration.sum","ns","54,000"
+"2","123","python3","127.0.0.1","void wmkv::(anonymous namespace)::attend_kernel<64>(wmkv::(anonymous namespace)::AttendParams)","1","7","(384, 1, 1)","(9, 16, 1)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","B","29,050,000"
 "2","123","python3","127.0.0.1","void wmkv::(anonymous namespace)::attend_kernel<64>(wmkv::(anonymous namespace)::AttendParams)","1","7","(384, 1, 1)","(9, 16, 1)","0","10.0","Command line profiler metrics","dram__bytes_write.sum","byte","8000"
 '''
 

@@ -128,8 +128,10 @@ def test_served_single_block_steady_state(wm):
 DENSE_CASES = [(1, 1, 1, 64), (5, 3, 2, 64), (128, 128, 2, 64), (129, 300, 3, 64),
                (200, 129, 2, 64), (64, 1000, 1, 64), (300, 1000, 2, 128), (257, 129, 4, 128),
                (33, 1, 2, 128), (1104, 6528, 2, 64),
-               # key counts around the 96-key tiles of the d = 64 kernel
-               (130, 96, 2, 64), (130, 97, 2, 64), (130, 192, 1, 64), (130, 289, 2, 64)]
+               # key counts just below, at and above multiples of the 128-key tiles,
+               # and around 96 (a partly filled first tile)
+               (130, 96, 2, 64), (130, 97, 2, 64), (130, 127, 1, 64), (130, 256, 1, 64),
+               (130, 257, 2, 64), (130, 289, 2, 64)]
 
 
 def dense_inputs(lq, lk, heads, d, tag):
@@ -211,8 +213,8 @@ def test_sampled_rows_helper_is_in_range():
     (Layout(24, 42, 96, 2, 24, heads=4, d=64), range(30)),
     (Layout(3, 5, 2, 0, 4, heads=2, d=64), range(9)),
     (Layout(5, 7, 9, 2, 9, heads=2, d=128), range(14)),
-    # record and summary lengths multiples of 8: tiles run across the seams
-    # between the three key segments (short last tiles fall back)
+    # record and summary lengths multiples of 8: each of the three key segments
+    # ends in a partly filled tile whose missing rows are masked
     (Layout(4, 4, 8, 2, 6, heads=2, d=64), range(12)),
     (Layout(8, 10, 16, 1, 7, heads=2, d=64), range(14)),
 ])
