@@ -104,7 +104,7 @@ def test_fp8_served_single_block_steady_state(wm):
         kv.write_record(0, t, dev(k), dev(v))
         mem.write_record(0, t, k, v)
     check_codes(kv, mem)
-    sat = np.abs(dequantize_e4m3(mem.K[0, :, :1], ks[0, :1])) == np.float32(1 / 200) * 448
+    sat = (mem.K[0, :, 0] & 0x7F) == 0x7E                   # +-448: saturated codes of head 0
     assert sat.sum() > 1000                                 # saturation is exercised
     q, _, _ = si.record_inputs(51, 0, 0, 31, 1, L.R, L.heads, L.d)
     o = nan_out(L)

@@ -69,9 +69,9 @@ def test_wait_runs_out_then_handle_recovers(wm, L, fused):
     if fused:
         # the slot the timed-out launch was writing is undefined: write it again
         kv.write_attend(0, t, dev(q), dev(k), dev(v), o)
+        mem.write_record(0, t, k, v)
     else:
         kv.attend(0, dev(q), o)
-    mem.write_record(0, t, k, v)
     assert _status(kv, wm) == wm.WM_OK
     kd, vd = kv.kv_views(0)
     assert np.array_equal(host_bits(kd), mem.K[0]) and np.array_equal(host_bits(vd), mem.V[0])
