@@ -24,12 +24,10 @@
 // Pipeline per warpgroup g and its tile j (= g, g+2, ...):
 //   wait S_full[g] -> load the S row into registers -> arrive S_free[g]
 //   (for d = 64, P has its own TMEM columns, so the MMA warp can already issue
-//   S_{j+2} into S_g while this tile's softmax runs) -> p = 2^(s*log2(e)/sqrt(d)
-//   - m) in registers (MUFU, part on the FMA pipe), where the exponent
-//   reference m is the row max of the warpgroup's first tile and stays put
-//   until a tile's exponentials would reach 2^16 (then that tile is redone
-//   with m raised to its max; the final division by l is exact either way), so
-//   no row max precedes the exponentials -> wait O_done[g] (P.V
+//   S_{j+2} into S_g while this tile's softmax runs) -> row max; the exponent
+//   reference m moves only when the max grows by more than 2^8 (the final
+//   division by l is exact either way) -> p = 2^(s*log2(e)/sqrt(d) - m) in
+//   registers (MUFU, part on the FMA pipe) -> wait O_done[g] (P.V
 //   of tile j-2 finished: O_g is stable and P_g is free; waiting only now
 //   hides the MMA round trip behind the exponentials) -> rescale O_g if m
 //   moved -> P as bf16 into TMEM -> arrive P_full[g].
@@ -150,11 +148,9 @@ constexpr int poly_pairs_per_8() {
   return WMKV_POLY_PAIRS_PER_8 >= 0 ? WMKV_POLY_PAIRS_PER_8 : (D == 64 ? 3 : 0);
 }
 
-// Exponentials of a tile stay below 2^REF_HEADROOM (log2 units above the
-// reference): enough room that a stale reference rarely needs a redo, small
-// enough that p * v cannot overflow float32 for any |v| below 2^80.
-constexpr float REF_HEADROOM = 16.f;
-constexpr float REF_HEADROOM_EXP = 65536.f;  // 2^REF_HEADROOM
+// log2 units: O and l are rescaled only when the row max grows by more than
+// 2^8, so every exponential of a tile lies in (0, 2^8].
+constexpr float RESCALE_THRESHOLD = 8.f;
 
 // Largest of the 128 scores of a row: eight independent chains of
 // three-input max, then a tree.
@@ -171,20 +167,15 @@ __device__ __forceinline__ float row_max(const float (&s)[128]) {
   return fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], fmax3(mx[5], mx[6], mx[7])));
 }
 
-// p = 2^(s * sl2 - m_ref) for the 128 scores of a row, packed to bf16 pairs,
-// and their sum.  POLY of every 8 column pairs take the FMA-pipe polynomial,
-// the rest MUFU.EX2.  Returns false if some exponential may have reached
-// 2^REF_HEADROOM: for MUFU lanes the sum shows it (it would be at least that
-// large, or not finite), for polynomial lanes the largest argument (the
-// polynomial's bit arithmetic is only valid below 2^128).  NaN scores make it
-// return false as well.
+// p = 2^(s * sl2 - m_ref) for the 128 scores of a row, packed to bf16 pairs;
+// returns their sum.  POLY of every 8 column pairs take the FMA-pipe
+// polynomial, the rest MUFU.EX2 (the arguments are at most RESCALE_THRESHOLD).
 template <int POLY>
-__device__ __forceinline__ bool exp_tile(const float (&s)[128], float sl2, float m_ref,
-                                         uint32_t (&pk)[64], float& sum) {
+__device__ __forceinline__ float exp_tile(const float (&s)[128], float sl2, float m_ref,
+                                          uint32_t (&pk)[64]) {
   const f2 scale2 = f2_make(sl2, sl2);
   const f2 negm2 = f2_make(-m_ref, -m_ref);
   f2 acc0 = f2_make(0.f, 0.f), acc1 = acc0, acc2 = acc0, acc3 = acc0;
-  float xm[3] = {-INFINITY, -INFINITY, -INFINITY};  // largest polynomial-lane argument
 #pragma unroll
   for (int pp = 0; pp < 64; ++pp) {
     const f2 x = f2_fma(f2_make(s[2 * pp], s[2 * pp + 1]), scale2, negm2);
@@ -192,10 +183,6 @@ __device__ __forceinline__ bool exp_tile(const float (&s)[128], float sl2, float
     if (EXP_F16X2) {
       e = exp2_f16x2(x);
     } else if ((pp % 8) >= 8 - POLY) {
-      float x0, x1;
-      f2_split(x, x0, x1);
-      float& m = xm[(pp % 8) % 3];
-      m = fmax3(m, x0, x1);
       e = exp2_poly2(x);
     } else {
       float x0, x1;
@@ -215,9 +202,7 @@ __device__ __forceinline__ bool exp_tile(const float (&s)[128], float sl2, float
   const f2 acc = f2_add(f2_add(acc0, acc1), f2_add(acc2, acc3));
   float a_lo, a_hi;
   f2_split(acc, a_lo, a_hi);
-  sum = a_lo + a_hi;
-  const bool poly_ok = POLY == 0 || fmax3(xm[0], xm[1], xm[2]) < REF_HEADROOM;
-  return sum < REF_HEADROOM_EXP && poly_ok;
+  return a_lo + a_hi;
 }
 
 // The softmax warps tell the MMA issuers that a warpgroup has read S or
@@ -631,26 +616,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
             if (c >= valid) s[c] = -INFINITY;
         }
       }
-      // Exponent reference m_ref (log2 units).  The first tile of a warpgroup
-      // takes its row max; later tiles keep the reference of the earlier ones
-      // (the softmax does not depend on the reference: l and O carry the same
-      // factor and the final division removes it), so a tile's exponentials do
-      // not wait for its max.  A tile whose exponentials could reach
-      // 2^REF_HEADROOM -- some score far above the reference -- is caught
-      // afterwards by exp_tile and redone from the scores still in registers,
-      // with the reference raised to the tile's max (O and l rescaled).
+      // Exponent reference m_ref (log2 units): it moves only when the row max
+      // grows by more than RESCALE_THRESHOLD (then O and l are rescaled); the
+      // final division by l removes whatever reference was used.
+      const float m_tile = row_max(s) * sl2;
       float alpha = 1.f;
       bool grow = false;
-      if (n == 0) m_ref = row_max(s) * sl2;
-      uint32_t pk[64];
-      float tile_sum;
-      if (!exp_tile<poly_pairs_per_8<D>()>(s, sl2, m_ref, pk, tile_sum)) {
-        const float m_new = fmaxf(row_max(s) * sl2, m_ref);
-        alpha = ex2_approx(m_ref - m_new);
-        m_ref = m_new;
+      if (n == 0) {
+        m_ref = m_tile;
+      } else if (m_tile > m_ref + RESCALE_THRESHOLD) {
+        alpha = ex2_approx(m_ref - m_tile);
+        m_ref = m_tile;
         grow = true;
-        exp_tile<poly_pairs_per_8<D>()>(s, sl2, m_ref, pk, tile_sum);
       }
+      uint32_t pk[64];
+      const float tile_sum = exp_tile<poly_pairs_per_8<D>()>(s, sl2, m_ref, pk);
       // l is rescaled by alpha (1 unless the reference grew) before this tile's sum
       l_run = l_run * alpha + tile_sum;
       if (n > 0) {

@@ -344,7 +344,7 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 }
 
 // 2^x on the FMA pipe for x in [-125, 127] (softmax exponents: the attention
-// keeps them below 2^16 and checks that it did).  Cody-Waite style
+// keeps them at most 8, the lazy-rescale threshold).  Cody-Waite style
 // reduction x = j + f with j = round(x), f in [-1/2, 1/2] (W. J. Cody and
 // W. Waite, "Software Manual for the Elementary Functions", 1980): j is read
 // from the low mantissa bits of x + 1.5*2^23, 2^f is a minimax polynomial
