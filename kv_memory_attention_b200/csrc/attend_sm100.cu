@@ -167,6 +167,22 @@ __device__ __forceinline__ float row_max(const float (&s)[128]) {
   return fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], fmax3(mx[5], mx[6], mx[7])));
 }
 
+// Independent partial sums of a row's exponentials (a power of two).
+#ifndef WMKV_ACC_CHAINS
+#define WMKV_ACC_CHAINS 4
+#endif
+constexpr int ACC_CHAINS = WMKV_ACC_CHAINS;
+// Which of every 8 column pairs take the polynomial: the last POLY of each
+// group, or (WMKV_POLY_SPREAD) POLY spread through the group.
+#ifndef WMKV_POLY_SPREAD
+#define WMKV_POLY_SPREAD 0
+#endif
+template <int POLY>
+__device__ __forceinline__ constexpr bool poly_pair(int pp) {
+  return WMKV_POLY_SPREAD && POLY == 3 ? ((pp % 8) == 1 || (pp % 8) == 4 || (pp % 8) == 6)
+                                        : (pp % 8) >= 8 - POLY;
+}
+
 // p = 2^(s * sl2 - m_ref) for the 128 scores of a row, packed to bf16 pairs;
 // returns their sum.  POLY of every 8 column pairs take the FMA-pipe
 // polynomial, the rest MUFU.EX2 (the arguments are at most RESCALE_THRESHOLD).
@@ -175,33 +191,33 @@ __device__ __forceinline__ float exp_tile(const float (&s)[128], float sl2, floa
                                           uint32_t (&pk)[64]) {
   const f2 scale2 = f2_make(sl2, sl2);
   const f2 negm2 = f2_make(-m_ref, -m_ref);
-  f2 acc0 = f2_make(0.f, 0.f), acc1 = acc0, acc2 = acc0, acc3 = acc0;
+  f2 acc[ACC_CHAINS];
+#pragma unroll
+  for (int i = 0; i < ACC_CHAINS; ++i) acc[i] = f2_make(0.f, 0.f);
 #pragma unroll
   for (int pp = 0; pp < 64; ++pp) {
     const f2 x = f2_fma(f2_make(s[2 * pp], s[2 * pp + 1]), scale2, negm2);
     f2 e;
     if (EXP_F16X2) {
       e = exp2_f16x2(x);
-    } else if ((pp % 8) >= 8 - POLY) {
+    } else if (poly_pair<POLY>(pp)) {
       e = exp2_poly2(x);
     } else {
       float x0, x1;
       f2_split(x, x0, x1);
       e = f2_make(ex2_approx(x0), ex2_approx(x1));
     }
-    switch (pp % 4) {
-      case 0: acc0 = f2_add(acc0, e); break;
-      case 1: acc1 = f2_add(acc1, e); break;
-      case 2: acc2 = f2_add(acc2, e); break;
-      default: acc3 = f2_add(acc3, e); break;
-    }
+    acc[pp % ACC_CHAINS] = f2_add(acc[pp % ACC_CHAINS], e);
     float e0, e1;
     f2_split(e, e0, e1);
     pk[pp] = pack_bf16x2(e0, e1);
   }
-  const f2 acc = f2_add(f2_add(acc0, acc1), f2_add(acc2, acc3));
+#pragma unroll
+  for (int w = ACC_CHAINS / 2; w >= 1; w /= 2)
+#pragma unroll
+    for (int i = 0; i < w; ++i) acc[i] = f2_add(acc[i], acc[i + w]);
   float a_lo, a_hi;
-  f2_split(acc, a_lo, a_hi);
+  f2_split(acc[0], a_lo, a_hi);
   return a_lo + a_hi;
 }
 
