@@ -262,6 +262,35 @@ WM_API int wm_attend_dense_fp8(const void* Q, const void* K8, const void* V8, co
  * arguments it rejects). */
 WM_API int64_t wm_attend_dense_fp8_scratch_bytes(int64_t Lk, int heads, int d);
 
+/* wm_attend_dense_fp8 for callers that cannot allocate device memory.  The
+ * page has no counterpart: this entry point exists for callers that cannot
+ * hand wm_attend_dense_fp8 a scratch buffer -- a plug-in that receives only
+ * the tensors of one call and has no allocator, a host framework whose memory
+ * pool owns every device allocation and refuses outside ones, a serving
+ * process that must not grow its device footprint (or synchronise inside
+ * cudaMalloc / cudaFree) once it runs.  It computes exactly what
+ * wm_attend_dense_fp8 computes, with the same arguments minus the scratch:
+ * the keys and values are widened into a fixed device array of
+ * WM_FP8_STATIC_SCRATCH_BYTES (32 MiB) that this library defines and every
+ * GPU that loads the library holds until the process exits.  It calls no
+ * cudaMalloc, cudaFree or allocating library routine.
+ *   - Limit: 2 * Lk * heads * d * 2 bytes must fit the array (Lk * heads * d
+ *     at most 8,388,608, e.g. 6,528 keys x 16 heads x 64); larger calls
+ *     return WM_ERR_INVALID_ARG and launch nothing.
+ *   - The first call on a device looks up the array's device address with
+ *     that device current (once per device); make that first call before any
+ *     stream capture.
+ *   - Every call shares the one array.  Each call writes the part it reads
+ *     before reading it, so nothing needs clearing between calls, but calls
+ *     whose work overlaps on the GPU (other streams, other threads) race:
+ *     order them on one stream or with events.
+ * Other arguments, requirements and errors as for wm_attend_dense_fp8. */
+#define WM_FP8_STATIC_SCRATCH_BYTES (32ll << 20)
+WM_API int wm_attend_dense_fp8_static(const void* Q, const void* K8, const void* V8,
+                                      const float* k_scale, const float* v_scale, void* O,
+                                      int64_t Lq, int64_t Lk, int heads, int d, int* dev_status,
+                                      wm_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -96,6 +96,12 @@ int64_t record_row(int64_t hw, int64_t X, int64_t Y, int64_t t) {
 
 }  // namespace
 
+namespace wmkv {
+// Records a CUDA error for wm_last_cuda_error and returns WM_ERR_CUDA (for
+// entry points defined in other files).
+int note_cuda_error(cudaError_t e) { return cuda_fail(e); }
+}  // namespace wmkv
+
 extern "C" {
 
 static int kvbuf_create(wm_kvbuf** out, int blocks, int heads, int d, int grid_h, int grid_w, int X,

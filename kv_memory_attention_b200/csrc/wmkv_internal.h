@@ -68,6 +68,9 @@ cudaError_t launch_attend(const void* q, void* o, int64_t lq, const KVSegment* s
                           const float* v_scale, cudaStream_t stream);
 bool attend_copies_in_kernel(int d);
 
+// Keeps the CUDA error's text for wm_last_cuda_error; returns WM_ERR_CUDA.
+int note_cuda_error(cudaError_t e);
+
 // SM count of the current device (queried once per device).
 int device_sm_count();
 

@@ -59,7 +59,11 @@ SIGNATURES = {
     "wm_attend_dense_fp8": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _c_i64, _c_i64, _c_int, _c_int,
                                      _vp, _c_i64, _vp, _vp]),
     "wm_attend_dense_fp8_scratch_bytes": (_c_i64, [_c_i64, _c_int, _c_int]),
+    "wm_attend_dense_fp8_static": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _c_i64, _c_i64, _c_int,
+                                            _c_int, _vp, _vp]),
 }
+
+WM_FP8_STATIC_SCRATCH_BYTES = 32 << 20
 
 WM_KV_BF16 = 0
 WM_KV_E4M3 = 1
@@ -234,6 +238,14 @@ def wm_attend_dense_fp8(Q, K8, V8, k_scale, v_scale, O, Lq: int, Lk: int, heads:
     _check(LIB.wm_attend_dense_fp8(_ptr(Q), _ptr(K8), _ptr(V8), _ptr(k_scale), _ptr(v_scale), _ptr(O),
                                    Lq, Lk, heads, d, _ptr(scratch), scratch_bytes, _ptr(dev_status),
                                    _stream(stream)), "wm_attend_dense_fp8")
+
+
+def wm_attend_dense_fp8_static(Q, K8, V8, k_scale, v_scale, O, Lq: int, Lk: int, heads: int, d: int,
+                               dev_status=None, stream=None) -> None:
+    """wm_attend_dense_fp8 with the library's fixed device scratch (no allocation)."""
+    _check(LIB.wm_attend_dense_fp8_static(_ptr(Q), _ptr(K8), _ptr(V8), _ptr(k_scale), _ptr(v_scale),
+                                          _ptr(O), Lq, Lk, heads, d, _ptr(dev_status), _stream(stream)),
+           "wm_attend_dense_fp8_static")
 
 
 def wm_layout_capacity(grid_h, grid_w, X, Y, W) -> int:
