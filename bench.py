@@ -76,8 +76,9 @@ PROFILES = os.path.join(ROOT, "profiles")
 TRAFFIC_JSON = os.path.join(PROFILES, "attend_kernel_served.json")
 LAUNCHES_JSON = os.path.join(PROFILES, "frame_step_launches_served.json")
 CSRC = os.path.join(ROOT, "kv_memory_attention_b200", "csrc")
-# the files the attention kernel is compiled from
+# the files each kernel is compiled from
 ATTEND_SOURCES = ("attend_sm100.cu", "sm100_ptx.cuh", "wmkv_internal.h")
+COPY_SOURCES = ("copy_kernels.cu", "sm100_ptx.cuh", "wmkv_internal.h")
 
 
 def config_dict(world: int) -> dict:
@@ -101,13 +102,22 @@ def peaks() -> dict:
         return {"sustained": 1400.0, "burst": 1590.0, "hbm": 6650.0, "source": "fallback"}
 
 
-def source_digest() -> str:
-    """sha256 prefix of the attention kernel's source files (in a fixed order)."""
+def source_digest(files=ATTEND_SOURCES) -> str:
+    """sha256 prefix of a kernel's source files (in a fixed order)."""
     h = hashlib.sha256()
-    for name in ATTEND_SOURCES:
+    for name in files:
         with open(os.path.join(CSRC, name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
+
+
+def file_digests() -> dict:
+    """sha256 prefix of every library source file."""
+    out = {}
+    for name in sorted(os.listdir(CSRC)):
+        with open(os.path.join(CSRC, name), "rb") as f:
+            out[name] = hashlib.sha256(f.read()).hexdigest()[:16]
+    return out
 
 
 # ---------------------------------------------------------------- ncu summaries
@@ -176,18 +186,19 @@ def summarize_ncu_csv(path: str, command: str) -> dict:
         if rd is not None and wr is not None:
             entry["dram_bytes_per_launch"] = int(round((rd + wr) / n))
         kernels.append(entry)
-    return {"command": command, "source_sha256": source_digest(),
+    return {"command": command, "source_sha256": source_digest(), "sources": file_digests(),
             "captured_launches": len(launches), "kernels": kernels,
             "note": "ncu replays each launch cold and serialised: compare shares, not absolute times"}
 
 
-def _profile_entry(path: str, prefix: str):
-    """The kernel entry whose name starts with ``prefix`` in a summary JSON that
-    was taken from the current attention sources, else None."""
+def _profile_entry(path: str, prefix: str, files=ATTEND_SOURCES):
+    """The kernel entry whose name starts with ``prefix`` in a summary JSON
+    captured from the current version of ``files``, else None."""
     try:
         with open(path) as f:
             j = json.load(f)
-        if j.get("source_sha256") != source_digest():
+        now = file_digests()
+        if any(j.get("sources", {}).get(name) != now[name] for name in files):
             return None
         for k in j["kernels"]:
             if k["kernel"].startswith(prefix):
@@ -674,10 +685,16 @@ def extra_copies(torch, kv, t, K, V, hbm_gbs):
         return {"kernel": kernel, "bytes": nbytes, "us": round(us, 2), "GB_per_s": round(gbs, 1),
                 "frac_of_hbm": round(gbs / hbm_gbs, 3)}
 
-    return {"evict": entry("evict_kernel (28 blocks, one launch)", EVICT_BYTES, evict_us),
-            "record_write": entry("copy_pair_kernel (one block)", WRITE_BYTES, write_us),
-            "how": f"median of {n} launches, each after a 512 MB read (L2 holds no copy data); "
-                   "bytes = algorithmic read + write; CUDA events around one launch"}, t
+    out = {"evict": entry("evict_kernel (28 blocks, one launch)", EVICT_BYTES, evict_us),
+           "record_write": entry("copy_pair_kernel (one block)", WRITE_BYTES, write_us),
+           "how": f"median of {n} launches, each after a 512 MB read (L2 holds no copy data); "
+                  "bytes = algorithmic read + write; CUDA events around one launch, so launch "
+                  "and event overhead are included (an upper bound on the kernel's time)"}
+    ev = _profile_entry(LAUNCHES_JSON, "evict_kernel", COPY_SOURCES)
+    if ev is not None:
+        out["evict_ncu"] = entry("evict_kernel, ncu gpu__time_duration in the frame-step launch list",
+                                 EVICT_BYTES, ev["avg_us"])
+    return out, t
 
 
 def extra_batch(torch, wm, window, device, sessions=8, steps=20):

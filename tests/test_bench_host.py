@@ -75,9 +75,13 @@ def test_profile_entries_follow_the_source_digest(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "TRAFFIC_JSON", str(out))
     assert bench.load_traffic() == 29058000
     j = json.load(open(out))
-    j["source_sha256"] = "0" * 16                  # taken from other sources: stale
+    j["sources"]["attend_sm100.cu"] = "0" * 16     # taken from another version: stale
     json.dump(j, open(out, "w"))
     assert bench.load_traffic() is None
+    j["sources"]["attend_sm100.cu"] = bench.file_digests()["attend_sm100.cu"]
+    j["sources"]["copy_kernels.cu"] = "0" * 16     # the copy kernels do not feed the attention entry
+    json.dump(j, open(out, "w"))
+    assert bench.load_traffic() == 29058000
 
 
 def test_attention_launch_time_and_peak_choice():
