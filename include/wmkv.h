@@ -214,6 +214,15 @@ WM_API const char* wm_strerror(int code);
 /* Text of the last CUDA error seen by this thread in a wm_* call ("" if none). */
 WM_API const char* wm_last_cuda_error(void);
 
+/* Self-check of the polynomial 2^x the attention kernel evaluates on the FMA
+ * pipe for 3 of every 8 exponentials (head dimension 64): y[i] = that
+ * polynomial's 2^x[i], for device float arrays of n (even, >= 2) values,
+ * 8-byte aligned.  The page has no counterpart; the call exists so that a
+ * test can bound the approximation's error on the device (relative error at
+ * most 1.7e-3 for x in [-125, 127]; x below -125 gives 2^-125).
+ * WM_ERR_INVALID_ARG for NULL, misaligned or odd-sized arrays. */
+WM_API int wm_selftest_exp2(const float* x, float* y, int64_t n, wm_stream_t stream);
+
 /* Pure layout arithmetic (no handle, no device) used by tests and tools. */
 WM_API int64_t wm_layout_capacity(int grid_h, int grid_w, int X, int Y, int W);
 WM_API int64_t wm_layout_end(int grid_h, int grid_w, int X, int Y, int W, int64_t t);

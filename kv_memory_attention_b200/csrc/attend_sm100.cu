@@ -131,21 +131,11 @@ struct Cfg {
 
 // Of every 8 column pairs of a score row, this many get their exponential
 // from the FMA-pipe polynomial instead of MUFU.EX2 (measured on B200: 3 is
-// best for d = 64, where exponentials per FLOP are twice as frequent; 0 for
-// d = 128).
-#ifndef WMKV_POLY_PAIRS_PER_8
-#define WMKV_POLY_PAIRS_PER_8 -1
-#endif
-// Exponentials two per MUFU instruction in f16 (argument and result), widened
-// to f32 for the row sum and packed to bf16 for P.V.
-#ifndef WMKV_EXP_F16X2
-#define WMKV_EXP_F16X2 0
-#endif
-constexpr bool EXP_F16X2 = WMKV_EXP_F16X2 != 0;
-
+// best for d = 64, where exponentials per FLOP are twice as frequent, against
+// 2 and 4; 0 for d = 128).
 template <int D>
 constexpr int poly_pairs_per_8() {
-  return WMKV_POLY_PAIRS_PER_8 >= 0 ? WMKV_POLY_PAIRS_PER_8 : (D == 64 ? 3 : 0);
+  return D == 64 ? 3 : 0;
 }
 
 // log2 units: O and l are rescaled only when the row max grows by more than
@@ -167,21 +157,9 @@ __device__ __forceinline__ float row_max(const float (&s)[128]) {
   return fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], fmax3(mx[5], mx[6], mx[7])));
 }
 
-// Independent partial sums of a row's exponentials (a power of two).
-#ifndef WMKV_ACC_CHAINS
-#define WMKV_ACC_CHAINS 4
-#endif
-constexpr int ACC_CHAINS = WMKV_ACC_CHAINS;
-// Which of every 8 column pairs take the polynomial: the last POLY of each
-// group, or (WMKV_POLY_SPREAD) POLY spread through the group.
-#ifndef WMKV_POLY_SPREAD
-#define WMKV_POLY_SPREAD 0
-#endif
-template <int POLY>
-__device__ __forceinline__ constexpr bool poly_pair(int pp) {
-  return WMKV_POLY_SPREAD && POLY == 3 ? ((pp % 8) == 1 || (pp % 8) == 4 || (pp % 8) == 6)
-                                        : (pp % 8) >= 8 - POLY;
-}
+// Independent partial sums of a row's exponentials (a power of two; 8
+// measured slower than 4).
+constexpr int ACC_CHAINS = 4;
 
 // p = 2^(s * sl2 - m_ref) for the 128 scores of a row, packed to bf16 pairs;
 // returns their sum.  POLY of every 8 column pairs take the FMA-pipe
@@ -198,9 +176,7 @@ __device__ __forceinline__ float exp_tile(const float (&s)[128], float sl2, floa
   for (int pp = 0; pp < 64; ++pp) {
     const f2 x = f2_fma(f2_make(s[2 * pp], s[2 * pp + 1]), scale2, negm2);
     f2 e;
-    if (EXP_F16X2) {
-      e = exp2_f16x2(x);
-    } else if (poly_pair<POLY>(pp)) {
+    if ((pp % 8) >= 8 - POLY) {
       e = exp2_poly2(x);
     } else {
       float x0, x1;
@@ -226,17 +202,10 @@ __device__ __forceinline__ float exp_tile(const float (&s)[128], float sl2, floa
 // warp have completed at tcgen05.wait (a warp-wide instruction), so after the
 // fence and a warp sync one lane can speak for the warp (4 arrivals per
 // warpgroup instead of 128).
-#ifndef WMKV_WARP_ARRIVE
-#define WMKV_WARP_ARRIVE 1
-#endif
-constexpr uint32_t SOFTMAX_ARRIVALS = WMKV_WARP_ARRIVE ? 4 : 128;
+constexpr uint32_t SOFTMAX_ARRIVALS = 4;
 __device__ __forceinline__ void softmax_arrive(uint32_t bar, int lane) {
-  if (WMKV_WARP_ARRIVE) {
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bar);
-  } else {
-    mbar_arrive(bar);
-  }
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
 }
 
 // Keys come in up to MAX_SEGS segments, each with its own K and V tensor

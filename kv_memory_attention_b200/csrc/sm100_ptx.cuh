@@ -347,18 +347,15 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // keeps them at most 8, the lazy-rescale threshold).  Cody-Waite style
 // reduction x = j + f with j = round(x), f in [-1/2, 1/2] (W. J. Cody and
 // W. Waite, "Software Manual for the Elementary Functions", 1980): j is read
-// from the low mantissa bits of x + 1.5*2^23, 2^f is a minimax polynomial
-// (coefficients fitted for this library by Remez exchange on the relative
-// error over [-1/2, 1/2]: cubic 7.5e-5 = 2^-13.7, quadratic 1.7e-3 = 2^-9.2,
-// the latter about the size of the bf16 rounding P gets anyway), and 2^j is
+// from the low mantissa bits of x + 1.5*2^23, 2^f is a quadratic minimax
+// polynomial (coefficients fitted for this library by Remez exchange on the
+// relative error over [-1/2, 1/2]: at most 1.7e-3 = 2^-9.2, about the size of
+// the bf16 rounding P gets anyway; wm_selftest_exp2 checks it), and 2^j is
 // added into the exponent field.  x is clamped at -125 so the result stays a
 // normal float; anything below 2^-125 is negligible next to the largest term
 // of a softmax row (at least 1).  Above 127 the exponent field overflows and
 // the result is meaningless, which the caller must rule out.  Two lanes per
 // call (f32x2).
-#ifndef WMKV_POLY_DEGREE
-#define WMKV_POLY_DEGREE 2
-#endif
 __device__ __forceinline__ f2 exp2_poly2(f2 x) {
   float x0, x1;
   f2_split(x, x0, x1);
@@ -368,36 +365,14 @@ __device__ __forceinline__ f2 exp2_poly2(f2 x) {
   const f2 t = f2_add(x, magic);                         // round(x) in the low mantissa bits
   const f2 jf = f2_add(t, nmagic);                       // round(x) as a float
   const f2 f = f2_fma(jf, f2_make(-1.f, -1.f), x);       // x - round(x), exact
-#if WMKV_POLY_DEGREE == 2
   f2 p = f2_fma(f, f2_make(0.23842893540859222f, 0.23842893540859222f),
                 f2_make(0.7034479975700378f, 0.7034479975700378f));
   p = f2_fma(p, f, f2_make(1.0004431009292603f, 1.0004431009292603f));
-#else
-  f2 p = f2_fma(f, f2_make(0.0551716685295105f, 0.0551716685295105f),
-                f2_make(0.2426111251115799f, 0.2426111251115799f));
-  p = f2_fma(p, f, f2_make(0.6932609677314758f, 0.6932609677314758f));
-  p = f2_fma(p, f, f2_make(0.9999280571937561f, 0.9999280571937561f));
-#endif
   float p0, p1, t0, t1;
   f2_split(p, p0, p1);
   f2_split(t, t0, t1);
   return f2_make(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
                  __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
-}
-
-// 2^x for two lanes with one MUFU instruction: x rounded to f16, result f16
-// (10-bit mantissa), widened back to f32.
-__device__ __forceinline__ f2 exp2_f16x2(f2 x) {
-  float x0, x1;
-  f2_split(x, x0, x1);
-  uint32_t xh, eh;
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(xh) : "f"(x1), "f"(x0));
-  asm("ex2.approx.f16x2 %0, %1;" : "=r"(eh) : "r"(xh));
-  float e0, e1;
-  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
-      : "=f"(e0), "=f"(e1)
-      : "r"(eh));
-  return f2_make(e0, e1);
 }
 
 // Pack two floats to bf16x2 (round to nearest even); `lo` lands in the low half.

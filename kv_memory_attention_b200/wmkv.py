@@ -50,6 +50,7 @@ SIGNATURES = {
     "wm_set_wait_limit": (_c_int, [_vp, ctypes.c_uint64]),
     "wm_strerror": (ctypes.c_char_p, [_c_int]),
     "wm_last_cuda_error": (ctypes.c_char_p, []),
+    "wm_selftest_exp2": (_c_int, [_vp, _vp, _c_i64, _vp]),
     "wm_layout_capacity": (_c_i64, [_c_int, _c_int, _c_int, _c_int, _c_int]),
     "wm_layout_end": (_c_i64, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_i64]),
     "wm_layout_raw_slot": (_c_int, [_c_int, _c_i64]),
@@ -246,6 +247,10 @@ def wm_attend_dense_fp8_static(Q, K8, V8, k_scale, v_scale, O, Lq: int, Lk: int,
     _check(LIB.wm_attend_dense_fp8_static(_ptr(Q), _ptr(K8), _ptr(V8), _ptr(k_scale), _ptr(v_scale),
                                           _ptr(O), Lq, Lk, heads, d, _ptr(dev_status), _stream(stream)),
            "wm_attend_dense_fp8_static")
+
+
+def wm_selftest_exp2(x, y, n: int, stream=None) -> None:
+    _check(LIB.wm_selftest_exp2(_ptr(x), _ptr(y), n, _stream(stream)), "wm_selftest_exp2")
 
 
 def wm_layout_capacity(grid_h, grid_w, X, Y, W) -> int:

@@ -88,6 +88,9 @@ def test_null_handle_and_pointer_errors(wm):
     assert lib.wm_attend(None, 0, 16, 16, None) == wm.WM_ERR_INVALID_ARG
     assert lib.wm_sync_status(None) == wm.WM_ERR_INVALID_ARG
     assert lib.wm_set_wait_limit(None, 5) == wm.WM_ERR_INVALID_ARG
+    assert lib.wm_selftest_exp2(None, 16, 2, None) == wm.WM_ERR_INVALID_ARG
+    assert lib.wm_selftest_exp2(16, 16, 3, None) == wm.WM_ERR_INVALID_ARG
+    assert lib.wm_selftest_exp2(12, 16, 2, None) == wm.WM_ERR_INVALID_ARG
     assert lib.wm_kvbuf_destroy(None) == wm.WM_ERR_INVALID_ARG
     assert lib.wm_end(None) == -1
     # dense: misaligned / null pointers and bad sizes never reach the device
