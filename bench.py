@@ -433,7 +433,8 @@ def run_ours(args, world, rank, local):
     long_run, extras = None, None
     if world == 1 and not args.no_extras:
         long_run, t = extra_runs(torch, kv, t, Q, K, V, O)
-        extras, t = run_extras(torch, wm, device, kv, t, Q, K, V, O, window)
+        extras, t = run_extras(torch, wm, device, kv, t, Q, K, V, O, window,
+                               elapsed_ms / args.steps)
 
     value = aggregate_throughput(args.steps, elapsed_ms, world)
     pk = peaks()
@@ -884,7 +885,47 @@ def extra_fp8(torch, wm, Q, K, V, O, steps=50):
             "how": "advance + 28 x write_attend on an E4M3 memory (quantise, widen, attend)"}
 
 
-def run_extras(torch, wm, device, kv, t, Q, K, V, O, window):
+def extra_served_dense(torch, wm, device, ms_step, pk, steps=3):
+    """The page's comparison at the served shape: the same span kept at full
+    resolution, (W + 2) x 1008 = 26,208 keys, attended by the frame's 1008 raw
+    queries in every block (wm_attend_dense, per-block windows of one random
+    pool per tensor), against the memory's frame-step measured above."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(0x5EED + 6)
+    lk = (W + 2) * HW
+    assert lk == 26208
+
+    def randn(*shape):
+        return torch.randn(*shape, generator=gen, device=device).to(torch.bfloat16)
+
+    qp, kp, vp = randn(HW + (BLOCKS - 1) * 64, HEADS, D), randn(lk + (BLOCKS - 1) * 512, HEADS, D), \
+        randn(lk + (BLOCKS - 1) * 512, HEADS, D)
+    q = [qp[b * 64:b * 64 + HW] for b in range(BLOCKS)]
+    k = [kp[b * 512:b * 512 + lk] for b in range(BLOCKS)]
+    v = [vp[b * 512:b * 512 + lk] for b in range(BLOCKS)]
+    o = torch.empty(HW, HEADS, D, dtype=torch.bfloat16, device=device)
+    st = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def step():
+        for b in range(BLOCKS):
+            wm.wm_attend_dense(q[b], k[b], v[b], o, HW, lk, HEADS, D, st)
+
+    step()
+    ms = _timed(torch, step, steps)
+    if int(st.item()) != 0:
+        raise RuntimeError("dense attention reported a device timeout")
+    flop = BLOCKS * 4 * HW * lk * D * HEADS
+    tf = flop / (ms * 1e-3) / 1e12
+    peak, name = choose_peak(pk, ms * steps / 1e3)
+    return {"ms_per_step": round(ms, 4), "frame_steps_per_s": round(1e3 / ms, 3), "tflops": round(tf, 1),
+            "frac_of_bf16_peak": round(tf / peak, 4), "peak": f"{name} ({pk['source']})",
+            "queries": HW, "keys": lk, "steps": steps,
+            "memory_speedup": round(ms / ms_step, 2),
+            "how": "28 x wm_attend_dense over (W+2) x 1008 keys against the timed frame-step "
+                   "(advance + 28 x write_attend over 6,528 keys)"}
+
+
+def run_extras(torch, wm, device, kv, t, Q, K, V, O, window, ms_step):
     """All secondary measurements; a section that fails reports its error."""
     pk = peaks()
     out = {}
@@ -893,6 +934,7 @@ def run_extras(torch, wm, device, kv, t, Q, K, V, O, window):
                      ("copy_kernels", lambda: extra_copies(torch, kv, t, K, V, pk["hbm"])),
                      ("batch8", lambda: (extra_batch(torch, wm, window, device), t)),
                      ("fp8_buffer", lambda: (extra_fp8(torch, wm, Q, K, V, O), t)),
+                     ("served_vs_dense", lambda: (extra_served_dense(torch, wm, device, ms_step, pk), t)),
                      ("scaled_vs_dense", lambda: (extra_scaled(torch, wm, device, pk), t))):
         try:
             out[name], t = fn()

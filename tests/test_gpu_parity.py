@@ -128,6 +128,8 @@ def test_served_single_block_steady_state(wm):
 DENSE_CASES = [(1, 1, 1, 64), (5, 3, 2, 64), (128, 128, 2, 64), (129, 300, 3, 64),
                (200, 129, 2, 64), (64, 1000, 1, 64), (300, 1000, 2, 128), (257, 129, 4, 128),
                (33, 1, 2, 128), (1104, 6528, 2, 64),
+               # the page's full-resolution comparison point: 1008 raw queries x 26,208 keys
+               (1008, 26208, 2, 64),
                # key counts just below, at and above multiples of the 128-key tiles,
                # and around 96 (a partly filled first tile)
                (130, 96, 2, 64), (130, 97, 2, 64), (130, 127, 1, 64), (130, 256, 1, 64),
