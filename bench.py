@@ -877,11 +877,33 @@ def extra_fp8(torch, wm, Q, K, V, O, steps=50):
         step()
     ms = _timed(torch, step, steps)
     kv8.sync_status()
+
+    # the widening pass: dense FP8 attention minus dense bf16 attention over the
+    # same 6,528 keys (the K/V codes of block 0's buffer, widened by the call)
+    k8, v8 = kv8.kv_views(0)
+    dev = K[0].device
+    scale = torch.full((HEADS,), 1 / 64, dtype=torch.float32, device=dev)
+    nbytes = wm.wm_attend_dense_fp8_scratch_bytes(C, HEADS, D)
+    scratch = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    kb = torch.empty(C, HEADS, D, dtype=torch.bfloat16, device=dev)
+    vb = torch.empty_like(kb)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    n = 20
+    ms8 = _timed(torch, lambda: wm.wm_attend_dense_fp8(Q[0], k8, v8, scale, scale, O[0], R, C, HEADS, D,
+                                                       scratch, nbytes, st), n)
+    ms16 = _timed(torch, lambda: wm.wm_attend_dense(Q[0], kb, vb, O[0], R, C,
+                                                    HEADS, D, st), n)
     kv8.close()
+    widen_us = (ms8 - ms16) * 1e3
+    widen_bytes = 2 * C * HEADS * D * (1 + 2)         # codes read, bf16 written, K and V
     return {"value": round(1e3 / ms, 3), "unit": UNIT, "ms_per_step": round(ms, 4), "steps": steps,
             "launches_per_step": 1 + 3 * BLOCKS,
             "buffer_bytes": 2 * BLOCKS * C * HEADS * D,
             "tflops_per_step": round(BLOCKS * ATTN_FLOP / (ms * 1e-3) / 1e12, 1),
+            "widen": {"us": round(widen_us, 2), "bytes": widen_bytes,
+                      "GB_per_s": round(widen_bytes / max(widen_us, 1e-3) / 1e3, 1),
+                      "how": f"wm_attend_dense_fp8 minus wm_attend_dense over {C} keys x {HEADS} x {D}, "
+                             f"{n} calls each, back to back"},
             "how": "advance + 28 x write_attend on an E4M3 memory (quantise, widen, attend)"}
 
 
