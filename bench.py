@@ -885,8 +885,8 @@ def extra_fp8(torch, wm, Q, K, V, O, steps=50):
     scale = torch.full((HEADS,), 1 / 64, dtype=torch.float32, device=dev)
     nbytes = wm.wm_attend_dense_fp8_scratch_bytes(C, HEADS, D)
     scratch = torch.empty(nbytes, dtype=torch.uint8, device=dev)
-    kb = torch.empty(C, HEADS, D, dtype=torch.bfloat16, device=dev)
-    vb = torch.empty_like(kb)
+    kb = torch.zeros(C, HEADS, D, dtype=torch.bfloat16, device=dev)
+    vb = torch.zeros_like(kb)
     st = torch.zeros(1, dtype=torch.int32, device=dev)
     n = 20
     ms8 = _timed(torch, lambda: wm.wm_attend_dense_fp8(Q[0], k8, v8, scale, scale, O[0], R, C, HEADS, D,
