@@ -243,15 +243,14 @@ struct TileLoc {
   int row;
   int valid;
 };
-template <int TN = BN>
 __device__ __forceinline__ TileLoc tile_loc(const AttendParams& p, int j) {
   int seg = 0;
 #pragma unroll
   for (int k = 0; k < MAX_SEGS - 1; ++k) seg += (k < p.nseg - 1 && j >= p.seg_tiles_end[k]) ? 1 : 0;
   const int first = seg ? p.seg_tiles_end[seg - 1] : 0;
-  const int row = (j - first) * TN;
+  const int row = (j - first) * BN;
   const int left = p.seg_rows[seg] - row;
-  return {seg, row, left < TN ? left : TN};
+  return {seg, row, left < BN ? left : BN};
 }
 
 __device__ __forceinline__ void record_timeout(int* status) {
@@ -711,456 +710,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
   }
 }
 
-// ----------------------------------------------------------------------------
-// Head dimension 64 with three softmax warpgroups on 64-key tiles.
-//
-// The two-warpgroup kernel above leaves each SM sub-partition two softmax
-// warps to hide the exponential stream's latencies.  Here every
-// sub-partition has three (warpgroups 0-2 take key tiles j = g mod 3, 64 keys
-// each), and each warpgroup has its own MMA-issuing thread: a single thread
-// issues one tcgen05.mma per ~150 cycles whatever its size, while separate
-// threads add up until the tensor pipe is full, so the 16 smaller MMAs per
-// 128 keys come from three threads in parallel.
-//   warps 0-11   softmax warpgroup g = warp / 4: S_g, P_g, O_g in TMEM
-//   warp 12      TMA producer (Q, K and V rings of 64-key tiles, record copy);
-//                owns the TMEM allocation
-//   warps 13-15  MMA issuer of warpgroup warp - 13: S_j = Q K_j^T as soon as
-//                its warpgroup has read S_{j-3}, then O_g += P_j V_j
-// TMEM (512 columns): S_g at 64 g (64 columns), P_g at 192 + 32 g (64 bf16
-// per row), O_g at 288 + 64 g; the three partial results are merged per row
-// at the end.  Registers: 512 threads at 128, split 152 for each softmax
-// thread (64 scores, 32 packed P) and 56 for the control warpgroup.
-namespace three {
-constexpr int QROWS = 128;
-constexpr int TN = 64;                 // keys per tile
-constexpr int THREADS = 512;
-constexpr int REGS_AT_LAUNCH = 128;
-constexpr int REGS_SOFTMAX = 152;
-constexpr int REGS_CONTROL = 56;
-static_assert(3 * 128 * REGS_SOFTMAX + 128 * REGS_CONTROL <= THREADS * REGS_AT_LAUNCH,
-              "register split exceeds the launch budget");
-constexpr int TILE_BYTES = TN * 128;   // 64 rows x 128 B
-constexpr int Q_BYTES = QROWS * 128;
-constexpr int NK = 9;
-constexpr int NV = 9;
-constexpr int K_AHEAD = 3;
-constexpr int Q_OFF = 0;
-constexpr int K_OFF = Q_OFF + Q_BYTES;
-constexpr int V_OFF = K_OFF + NK * TILE_BYTES;
-constexpr int COPY_CHUNK_BYTES = 16384;
-constexpr int COPY_OFF = V_OFF + NV * TILE_BYTES;
-constexpr int BAR_OFF = COPY_OFF + 2 * COPY_CHUNK_BYTES;
-constexpr int B_Q = 0;
-constexpr int B_KFULL = 1;
-constexpr int B_KEMPTY = B_KFULL + NK;
-constexpr int B_VFULL = B_KEMPTY + NK;
-constexpr int B_VEMPTY = B_VFULL + NV;
-constexpr int B_SFULL = B_VEMPTY + NV;  // 3
-constexpr int B_SFREE = B_SFULL + 3;    // 3
-constexpr int B_PFULL = B_SFREE + 3;    // 3
-constexpr int B_ODONE = B_PFULL + 3;    // 3
-constexpr int B_OFINAL = B_ODONE + 3;   // 1 barrier, 3 arrivals
-constexpr int B_DRAIN = B_OFINAL + 1;   // 3
-constexpr int B_COPY = B_DRAIN + 3;     // 2
-constexpr int NBAR = B_COPY + 2;
-constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
-constexpr int XCH_OFF = Q_OFF;           // m[3][128], l[3][128] after the last MMA
-constexpr int SMEM_BYTES = MISC_OFF + 16;
-constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
-static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory budget");
-constexpr uint32_t S_COL = 0;
-constexpr uint32_t P_COL = 192;
-constexpr uint32_t O_COL = 288;
-constexpr uint32_t TMEM_COLS = 512;
-static_assert(O_COL + 3 * 64 <= TMEM_COLS, "TMEM budget");
-constexpr uint32_t IDESC_S = idesc_bf16_f32(QROWS, TN, false, false);
-constexpr uint32_t IDESC_O = idesc_bf16_f32(QROWS, 64, false, true);
-constexpr int POLY = 3;                  // of every 8 column pairs on the FMA pipe
-}  // namespace three
-
-// Largest of 64 scores: eight chains of three-input max, then a tree.
-__device__ __forceinline__ float row_max64(const float (&s)[64]) {
-  float mx[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) mx[i] = fmax3(s[i], s[i + 8], s[i + 16]);
-#pragma unroll
-  for (int c = 24; c < 56; c += 16)
-#pragma unroll
-    for (int i = 0; i < 8; ++i) mx[i] = fmax3(mx[i], s[c + i], s[c + 8 + i]);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[56 + i]);
-  return fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], fmax3(mx[5], mx[6], mx[7])));
-}
-
-// p = 2^(s * sl2 - m_ref) for 64 scores, packed to bf16 pairs; returns their sum.
-__device__ __forceinline__ float exp_tile64(const float (&s)[64], float sl2, float m_ref,
-                                            uint32_t (&pk)[32]) {
-  const f2 scale2 = f2_make(sl2, sl2);
-  const f2 negm2 = f2_make(-m_ref, -m_ref);
-  f2 acc[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) acc[i] = f2_make(0.f, 0.f);
-#pragma unroll
-  for (int pp = 0; pp < 32; ++pp) {
-    const f2 x = f2_fma(f2_make(s[2 * pp], s[2 * pp + 1]), scale2, negm2);
-    f2 e;
-    if ((pp % 8) >= 8 - three::POLY) {
-      e = exp2_poly2(x);
-    } else {
-      float x0, x1;
-      f2_split(x, x0, x1);
-      e = f2_make(ex2_approx(x0), ex2_approx(x1));
-    }
-    acc[pp % 4] = f2_add(acc[pp % 4], e);
-    float e0, e1;
-    f2_split(e, e0, e1);
-    pk[pp] = pack_bf16x2(e0, e1);
-  }
-  const f2 a = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
-  float lo, hi;
-  f2_split(a, lo, hi);
-  return lo + hi;
-}
-
-__global__ void __launch_bounds__(three::THREADS, 1) attend3_kernel(const __grid_constant__ AttendParams p) {
-  using namespace three;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
-  const uint32_t sbase = smem_u32(smem);
-  auto bar = [&](int i) -> uint32_t { return sbase + BAR_OFF + 8 * i; };
-  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + MISC_OFF);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
-  float* xch_m = reinterpret_cast<float*>(smem + XCH_OFF);
-  float* xch_l = xch_m + 3 * QROWS;
-
-  const int warp = threadIdx.x / 32;
-  const int lane = threadIdx.x % 32;
-  const int q_tile = blockIdx.x;
-  const int head = blockIdx.y;
-  const int nkv = p.seg_tiles_end[p.nseg - 1];
-
-  pdl_launch_dependents();
-  if (threadIdx.x == 0) {
-    mbar_init(bar(B_Q), 1);
-    for (int s = 0; s < NK; ++s) {
-      mbar_init(bar(B_KFULL + s), 1);
-      mbar_init(bar(B_KEMPTY + s), 1);
-    }
-    for (int s = 0; s < NV; ++s) {
-      mbar_init(bar(B_VFULL + s), 1);
-      mbar_init(bar(B_VEMPTY + s), 1);
-    }
-    for (int g = 0; g < 3; ++g) {
-      mbar_init(bar(B_SFULL + g), 1);
-      mbar_init(bar(B_SFREE + g), SOFTMAX_ARRIVALS);
-      mbar_init(bar(B_PFULL + g), SOFTMAX_ARRIVALS);
-      mbar_init(bar(B_ODONE + g), 1);
-    }
-    mbar_init(bar(B_OFINAL), 3);  // each issuer commits once after its last P.V
-    for (int i = 0; i < 3; ++i) mbar_init(bar(B_DRAIN + i), 1);
-    mbar_init(bar(B_COPY), 1);
-    mbar_init(bar(B_COPY + 1), 1);
-    misc[1] = 0;
-    fence_mbar_init();
-  }
-  if (warp == 12) {
-    tmem_alloc(smem_u32(misc), TMEM_COLS);
-    tmem_relinquish();
-  }
-  if (warp == 12 && lane == 0) {
-    tma_prefetch_desc(&p.tm_q);
-    for (int k = 0; k < p.nseg; ++k) {
-      tma_prefetch_desc(&p.tm_k[k]);
-      tma_prefetch_desc(&p.tm_v[k]);
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = misc[0];
-  pdl_wait_prior();
-
-  if (warp >= 12) {
-    regs_dec<REGS_CONTROL>();
-    if (warp == 12) {
-      // ------------------------------------------------------------ producer
-      if (lane == 0) {
-        mbar_expect_tx(bar(B_Q), Q_BYTES);
-        tma_load_3d(sbase + Q_OFF, &p.tm_q, 0, head, q_tile * QROWS, bar(B_Q));
-        bool copied = p.copy_n16 <= 0;
-        auto copy_record = [&]() {
-          const int64_t G = int64_t(gridDim.x) * gridDim.y;
-          const int64_t c = int64_t(blockIdx.y) * gridDim.x + blockIdx.x;
-          const int64_t per = (p.copy_n16 + G - 1) / G;
-          const int64_t lo = c * per;
-          const int64_t hi = lo + per < p.copy_n16 ? lo + per : p.copy_n16;
-          constexpr int64_t CH = COPY_CHUNK_BYTES / 16;
-          uint32_t cph = 0;
-          for (int64_t u = lo; u < hi && !*abort_flag; u += CH) {
-            const uint32_t bytes = static_cast<uint32_t>((hi - u < CH ? hi - u : CH) * 16);
-            bulk_wait_read_all();
-            for (int t = 0; t < 2; ++t) {
-              mbar_expect_tx(bar(B_COPY + t), bytes);
-              bulk_load(sbase + COPY_OFF + t * COPY_CHUNK_BYTES, p.copy_src[t] + u, bytes,
-                        bar(B_COPY + t));
-            }
-            int landed = 0;
-            for (; landed < 2; ++landed) {
-              if (!mbar_wait_bounded(bar(B_COPY + landed), cph, abort_flag, p.wait_limit)) break;
-              bulk_store(p.copy_dst[landed] + u, sbase + COPY_OFF + landed * COPY_CHUNK_BYTES, bytes);
-            }
-            bulk_commit();
-            if (landed < 2) {
-              volatile int no_abort = 0;
-              for (int t = landed; t < 2; ++t)
-                mbar_wait_bounded(bar(B_COPY + t), cph, &no_abort, DRAIN_LIMIT_CYCLES);
-              break;
-            }
-            cph ^= 1;
-          }
-        };
-        int k_issued = 0, v_issued = 0;
-        for (int i = 0; i < nkv + K_AHEAD; ++i) {
-          if (!copied && (i >= NK || i >= nkv)) {
-            copy_record();
-            copied = true;
-          }
-          if (i < nkv) {
-            const int st = i % NK;
-            if (i >= NK && !mbar_wait_bounded(bar(B_KEMPTY + st), ((i / NK) - 1) & 1, abort_flag,
-                                              p.wait_limit))
-              break;
-            const TileLoc tl = tile_loc<TN>(p, i);
-            mbar_expect_tx(bar(B_KFULL + st), TILE_BYTES);
-            tma_load_3d(sbase + K_OFF + st * TILE_BYTES, &p.tm_k[tl.seg], 0, head, tl.row,
-                        bar(B_KFULL + st));
-            k_issued = i + 1;
-          }
-          const int jv = i - K_AHEAD;
-          if (jv >= 0 && jv < nkv) {
-            const int st = jv % NV;
-            if (jv >= NV && !mbar_wait_bounded(bar(B_VEMPTY + st), ((jv / NV) - 1) & 1, abort_flag,
-                                               p.wait_limit))
-              break;
-            const TileLoc tl = tile_loc<TN>(p, jv);
-            mbar_expect_tx(bar(B_VFULL + st), TILE_BYTES);
-            tma_load_3d(sbase + V_OFF + st * TILE_BYTES, &p.tm_v[tl.seg], 0, head, tl.row,
-                        bar(B_VFULL + st));
-            v_issued = jv + 1;
-          }
-        }
-        if (!copied) copy_record();
-        bulk_wait_all();
-        if (*abort_flag) {
-          volatile int no_abort = 0;
-          mbar_wait_bounded(bar(B_Q), 0, &no_abort, DRAIN_LIMIT_CYCLES);
-          for (int i = k_issued - NK < 0 ? 0 : k_issued - NK; i < k_issued; ++i)
-            mbar_wait_bounded(bar(B_KFULL + i % NK), (i / NK) & 1, &no_abort, DRAIN_LIMIT_CYCLES);
-          for (int i = v_issued - NV < 0 ? 0 : v_issued - NV; i < v_issued; ++i)
-            mbar_wait_bounded(bar(B_VFULL + i % NV), (i / NV) & 1, &no_abort, DRAIN_LIMIT_CYCLES);
-        }
-      }
-    } else if (lane == 0) {
-      // ------------------------------------------------------------ MMA issuer of warpgroup g
-      const int g = warp - 13;
-      const uint64_t dq = sdesc_sw128(sbase + Q_OFF, 16, 1024);
-      const uint64_t dk0 = sdesc_sw128(sbase + K_OFF, 16, 1024);
-      const uint64_t dv0 = sdesc_sw128(sbase + V_OFF, TILE_BYTES, 1024);
-      constexpr uint64_t TILE16 = TILE_BYTES >> 4;
-      const uint32_t s_tm = tmem + S_COL + 64 * g;
-      const uint32_t p_tm = tmem + P_COL + 32 * g;
-      const uint32_t o_tm = tmem + O_COL + 64 * g;
-      bool ok = mbar_spin_bounded(bar(B_Q), 0, abort_flag, p.wait_limit);
-      auto issue_s = [&](int j) -> bool {
-        const int st = j % NK;
-        if (!mbar_spin_bounded(bar(B_KFULL + st), (j / NK) & 1, abort_flag, p.wait_limit)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t off = uint64_t((kk * 32) >> 4);
-          mma_ss(s_tm, dq + off, dk0 + st * TILE16 + off, IDESC_S, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(bar(B_SFULL + g));
-        tc_commit(bar(B_KEMPTY + st));
-        return true;
-      };
-      if (ok && g < nkv) ok = issue_s(g);
-      int n = 0;
-      for (int j = g; ok && j < nkv; j += 3, ++n) {
-        if (j + 3 < nkv) {
-          // the warpgroup has read S_j: S_{j+3} may overwrite S_g
-          if (!mbar_wait_bounded(bar(B_SFREE + g), n & 1, abort_flag, p.wait_limit) ||
-              !issue_s(j + 3)) {
-            ok = false;
-            break;
-          }
-        }
-        const int vst = j % NV;
-        if (!mbar_wait_bounded(bar(B_PFULL + g), n & 1, abort_flag, p.wait_limit) ||
-            !mbar_spin_bounded(bar(B_VFULL + vst), (j / NV) & 1, abort_flag, p.wait_limit)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ts(o_tm, p_tm + kk * 8, dv0 + vst * TILE16 + uint64_t((kk * 2048) >> 4), IDESC_O,
-                 (n > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(bar(B_ODONE + g));
-        tc_commit(bar(B_VEMPTY + vst));
-      }
-      if (ok) {
-        tc_commit(bar(B_OFINAL));
-      } else {
-        volatile int no_abort = 0;
-        tc_commit(bar(B_DRAIN + g));
-        mbar_wait_bounded(bar(B_DRAIN + g), 0, &no_abort, DRAIN_LIMIT_CYCLES);
-      }
-    }
-  } else {
-    regs_inc<REGS_SOFTMAX>();
-    // ------------------------------------------------------------ softmax
-    const int g = warp / 4;
-    const int wq = warp % 4;
-    const int row = wq * 32 + lane;
-    const uint32_t lane_off = uint32_t(wq * 32) << 16;
-    const uint32_t s_addr = tmem + lane_off + S_COL + 64 * g;
-    const uint32_t p_addr = tmem + lane_off + P_COL + 32 * g;
-    const uint32_t o_addr = tmem + lane_off + O_COL + 64 * g;
-    const float sl2 = p.k_scale ? p.scale_log2 * p.k_scale[head] : p.scale_log2;
-    float m_ref = -INFINITY;
-    float l_run = 0.f;
-    bool ok = true;
-    int n = 0;
-    for (int j = g; j < nkv; j += 3, ++n) {
-      ok = mbar_wait_bounded(bar(B_SFULL + g), n & 1, abort_flag, p.wait_limit);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t sr[64];
-      tmem_ld32_at<0>(s_addr, sr);
-      tmem_ld32_at<32>(s_addr + 32, sr);
-      tmem_wait_ld();
-      tc_fence_before();
-      softmax_arrive(bar(B_SFREE + g), lane);
-      float s[64];
-#pragma unroll
-      for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sr[c]);
-      {
-        const int valid = tile_loc<TN>(p, j).valid;
-        if (valid < TN) {
-#pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (c >= valid) s[c] = -INFINITY;
-        }
-      }
-      const float m_tile = row_max64(s) * sl2;
-      float alpha = 1.f;
-      bool grow = false;
-      if (n == 0) {
-        m_ref = m_tile;
-      } else if (m_tile > m_ref + RESCALE_THRESHOLD) {
-        alpha = ex2_approx(m_ref - m_tile);
-        m_ref = m_tile;
-        grow = true;
-      }
-      uint32_t pk[32];
-      const float tile_sum = exp_tile64(s, sl2, m_ref, pk);
-      l_run = l_run * alpha + tile_sum;
-      if (n > 0) {
-        // P_{j-3}.V_{j-3} has finished: O_g is stable and P_g is free
-        ok = mbar_wait_bounded(bar(B_ODONE + g), (n - 1) & 1, abort_flag, p.wait_limit);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, grow)) {
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            uint32_t orr[32];
-            tmem_ld32(o_addr + c * 32, orr);
-            tmem_wait_ld();
-            const f2 a2 = f2_make(alpha, alpha);
-#pragma unroll
-            for (int i = 0; i < 32; i += 2) {
-              f2 v = f2_make(__uint_as_float(orr[i]), __uint_as_float(orr[i + 1]));
-              v = f2_mul(v, a2);
-              float lo, hi;
-              f2_split(v, lo, hi);
-              orr[i] = __float_as_uint(lo);
-              orr[i + 1] = __float_as_uint(hi);
-            }
-            tmem_st32(o_addr + c * 32, orr);
-          }
-        }
-      }
-      tmem_st32(p_addr, pk);
-      tmem_wait_st();
-      tc_fence_before();
-      softmax_arrive(bar(B_PFULL + g), lane);
-    }
-    if (ok) {
-      ok = mbar_wait_bounded(bar(B_OFINAL), 0, abort_flag, p.wait_limit);
-      ok = __all_sync(0xffffffffu, ok);
-    }
-    tc_fence_after();
-    xch_m[g * QROWS + row] = m_ref;
-    xch_l[g * QROWS + row] = l_run;
-    named_bar_sync(1, 384);
-    if (ok && !*abort_flag && g < 2) {
-      // warpgroup 0 stores columns 0-31, warpgroup 1 columns 32-63
-      const bool has1 = nkv > 1, has2 = nkv > 2;
-      const float m0 = xch_m[row], m1 = has1 ? xch_m[QROWS + row] : -INFINITY,
-                  m2 = has2 ? xch_m[2 * QROWS + row] : -INFINITY;
-      const float mf = fmax3(m0, m1, m2);
-      const float a0 = ex2_approx(m0 - mf);
-      const float a1 = has1 ? ex2_approx(m1 - mf) : 0.f;
-      const float a2 = has2 ? ex2_approx(m2 - mf) : 0.f;
-      const float l0 = xch_l[row], l1 = has1 ? xch_l[QROWS + row] : 0.f, l2 = has2 ? xch_l[2 * QROWS + row] : 0.f;
-      const float inv = (p.v_scale ? p.v_scale[head] : 1.f) / (l0 * a0 + l1 * a1 + l2 * a2);
-      const float c0 = a0 * inv, c1 = a1 * inv, c2 = a2 * inv;
-      const int col = 32 * g;
-      const uint32_t ob = tmem + lane_off + O_COL + col;
-      uint32_t r0[32], r1[32], r2[32];
-      tmem_ld32(ob, r0);
-      if (has1) tmem_ld32(ob + 64, r1);
-      if (has2) tmem_ld32(ob + 128, r2);
-      tmem_wait_ld();
-      uint32_t packed[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        float x0 = __uint_as_float(r0[2 * i]) * c0;
-        float x1 = __uint_as_float(r0[2 * i + 1]) * c0;
-        if (has1) {
-          x0 = fmaf(__uint_as_float(r1[2 * i]), c1, x0);
-          x1 = fmaf(__uint_as_float(r1[2 * i + 1]), c1, x1);
-        }
-        if (has2) {
-          x0 = fmaf(__uint_as_float(r2[2 * i]), c2, x0);
-          x1 = fmaf(__uint_as_float(r2[2 * i + 1]), c2, x1);
-        }
-        packed[i] = pack_bf16x2(x0, x1);
-      }
-      const int64_t qrow = int64_t(q_tile) * QROWS + row;
-      if (qrow < p.lq) {
-        uint4* dst = reinterpret_cast<uint4*>(p.o + (qrow * p.heads + head) * 64 + col);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
-      }
-    }
-  }
-
-  __syncwarp();
-  tc_fence_before();
-  __syncthreads();
-  if (threadIdx.x == 0 && *abort_flag) record_timeout(p.status);
-  if (warp == 12) {
-    tc_fence_after();
-    tmem_dealloc(tmem, three::TMEM_COLS);
-  }
-}
-
 // ---------------------------------------------------------------- host side
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
@@ -1177,14 +726,13 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
-// [rows, heads, d] bf16, box = box_rows rows x 1 head x 64 columns, 128-byte swizzle.
-bool encode_rows_map(CUtensorMap* m, const void* base, int64_t rows, int heads, int d,
-                     uint32_t box_rows = 128) {
+// [rows, heads, d] bf16, box = 128 rows x 1 head x 64 columns, 128-byte swizzle.
+bool encode_rows_map(CUtensorMap* m, const void* base, int64_t rows, int heads, int d) {
   auto enc = get_encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(heads), cuuint64_t(rows)};
   cuuint64_t strides[2] = {cuuint64_t(d) * 2, cuuint64_t(heads) * d * 2};
-  cuuint32_t box[3] = {64, 1, box_rows};
+  cuuint32_t box[3] = {64, 1, 128};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -1218,34 +766,6 @@ cudaError_t launch_d(const AttendParams& prm, int64_t lq, int heads, cudaStream_
   return launch_pdl(attend_kernel<D>, grid, dim3(NUM_THREADS), C::SMEM_ALLOC, stream, prm);
 }
 
-cudaError_t launch_three(const AttendParams& prm, int64_t lq, int heads, cudaStream_t stream) {
-  using namespace three;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES)
-    return cudaErrorInvalidDevice;
-  static std::once_flag once[MAX_DEVICES];
-  static cudaError_t attr_err[MAX_DEVICES];
-  std::call_once(once[dev], [dev] {
-    cudaError_t e = cudaFuncSetAttribute(attend3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         SMEM_ALLOC);
-    // setmaxnreg.inc waits until registers are free: the launch must carry
-    // exactly the budget the split assumes, or the kernel is not launched.
-    cudaFuncAttributes fa;
-    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, attend3_kernel);
-    if (e == cudaSuccess && fa.numRegs != REGS_AT_LAUNCH) e = cudaErrorInvalidConfiguration;
-    attr_err[dev] = e;
-  });
-  if (attr_err[dev] != cudaSuccess) return attr_err[dev];
-  dim3 grid(static_cast<unsigned>((lq + QROWS - 1) / QROWS), static_cast<unsigned>(heads));
-  return launch_pdl(attend3_kernel, grid, dim3(THREADS), SMEM_ALLOC, stream, prm);
-}
-
-// Head dimension 64 runs on the three-warpgroup kernel (64-key tiles).
-#ifndef WMKV_ATTEND3
-#define WMKV_ATTEND3 0
-#endif
-constexpr bool USE_THREE = WMKV_ATTEND3 != 0;
-
 }  // namespace
 
 bool attend_copies_in_kernel(int d) { return Cfg<64>::COPY_IN_KERNEL && d == 64; }
@@ -1255,17 +775,15 @@ cudaError_t launch_attend(const void* q, void* o, int64_t lq, const KVSegment* s
                           unsigned long long wait_limit, const float* k_scale,
                           const float* v_scale, cudaStream_t stream) {
   if (nseg < 1 || nseg > MAX_SEGS) return cudaErrorInvalidValue;
-  const bool three_wg = USE_THREE && d == 64;
-  const int tn = three_wg ? three::TN : BN;  // keys per tile
   AttendParams prm = {};
   if (!encode_rows_map(&prm.tm_q, q, lq, heads, d)) return cudaErrorInvalidValue;
   int tiles = 0;
   for (int k = 0; k < nseg; ++k) {
     if (segs[k].rows < 1 || segs[k].rows >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
-    if (!encode_rows_map(&prm.tm_k[k], segs[k].k, segs[k].rows, heads, d, tn) ||
-        !encode_rows_map(&prm.tm_v[k], segs[k].v, segs[k].rows, heads, d, tn))
+    if (!encode_rows_map(&prm.tm_k[k], segs[k].k, segs[k].rows, heads, d) ||
+        !encode_rows_map(&prm.tm_v[k], segs[k].v, segs[k].rows, heads, d))
       return cudaErrorInvalidValue;
-    tiles += static_cast<int>((segs[k].rows + tn - 1) / tn);
+    tiles += static_cast<int>((segs[k].rows + BN - 1) / BN);
     prm.seg_tiles_end[k] = tiles;
     prm.seg_rows[k] = static_cast<int>(segs[k].rows);
   }
@@ -1286,7 +804,6 @@ cudaError_t launch_attend(const void* q, void* o, int64_t lq, const KVSegment* s
     prm.copy_dst[1] = static_cast<uint4*>(copy->v_dst);
     prm.copy_n16 = copy->n16;
   }
-  if (three_wg) return launch_three(prm, lq, heads, stream);
   if (d == 64) return launch_d<64>(prm, lq, heads, stream);
   if (d == 128) return launch_d<128>(prm, lq, heads, stream);
   return cudaErrorInvalidValue;
