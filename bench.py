@@ -81,14 +81,32 @@ ATTEND_SOURCES = ("attend_sm100.cu", "sm100_ptx.cuh", "wmkv_internal.h")
 COPY_SOURCES = ("copy_kernels.cu", "sm100_ptx.cuh", "wmkv_internal.h")
 
 
-def config_dict(world: int) -> dict:
+# --kv-format e4m3: the same workload on the FP8 memory, one scale for every
+# (block, head) of K and of V (N(0,1) values stay well inside E4M3's range)
+FP8_SCALE = 1.0 / 64
+
+
+def config_dict(world: int, kv_format: str = "bf16") -> dict:
     """The workload, identical for both arms."""
-    return {"workload": WORKLOAD, "blocks": BLOCKS, "heads": HEADS, "head_dim": D,
-            "grid": f"{GH}x{GW}", "X": X, "Y": Y, "W": W, "queries": R, "keys": C,
-            "passes_per_frame": 1,
-            "parallelism": f"replicas x{world} (independent sessions)",
-            "l2": "no flush: per step the 28 blocks touch 748 MB of K/V buffers + 190 MB of "
-                  "inputs, far above the 126 MB L2"}
+    c = {"workload": WORKLOAD, "blocks": BLOCKS, "heads": HEADS, "head_dim": D,
+         "grid": f"{GH}x{GW}", "X": X, "Y": Y, "W": W, "queries": R, "keys": C,
+         "passes_per_frame": 1,
+         "parallelism": f"replicas x{world} (independent sessions)",
+         "l2": "no flush: per step the 28 blocks touch 748 MB of K/V buffers + 190 MB of "
+               "inputs, far above the 126 MB L2"}
+    if kv_format != "bf16":
+        c.update({"kv_format": kv_format, "kv_scale": FP8_SCALE,
+                  "l2": "no flush: per step the 28 blocks touch 374 MB of FP8 K/V buffers + 190 MB "
+                        "of inputs, far above the 126 MB L2"})
+    return c
+
+
+def make_memory(wm, kv_format: str, blocks=BLOCKS, heads=HEADS, d=D, gh=GH, gw=GW, x=X, y=Y, w=W):
+    if kv_format == "e4m3":
+        n = blocks * heads
+        return wm.KVMemory(blocks, heads, d, gh, gw, x, y, w, kv_format="e4m3",
+                           k_scale=[FP8_SCALE] * n, v_scale=[FP8_SCALE] * n)
+    return wm.KVMemory(blocks, heads, d, gh, gw, x, y, w)
 
 
 def peaks() -> dict:
@@ -339,11 +357,12 @@ def run_ours(args, world, rank, local):
 
     # CPU baseline (rank 0, N = 1): the oracle timed on host cores, and the GPU
     # path checked against it on the same inputs before anything is timed
+    fp8 = args.kv_format == "e4m3"
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline_and_parity(args.cpu_seconds, torch, wm)
+        cpu = cpu_baseline_and_parity(args.cpu_seconds, torch, wm, args.kv_format)
 
-    kv = wm.KVMemory(BLOCKS, HEADS, D, GH, GW, X, Y, W)
+    kv = make_memory(wm, args.kv_format)
     pool = torch.from_numpy(si._pool()["bf16"].view(np.int16)).to(device).view(torch.bfloat16)
     psize = pool.shape[0]
     n = R * HEADS * D
@@ -402,7 +421,7 @@ def run_ours(args, world, rank, local):
     barrier(world)
     kv.sync_status()
     elapsed_ms = max_over_ranks(start.elapsed_time(stop), world, device)
-    launches = args.steps * (1 + BLOCKS)
+    launches = args.steps * (1 + (3 if fp8 else 1) * BLOCKS)
 
     # ------------------------------------------------ attention launch time (roofline)
     # The same steps again with an event pair around each eviction only: the
@@ -431,7 +450,7 @@ def run_ours(args, world, rank, local):
 
     # ------------------------------------------------ longer runs and secondary measurements (N = 1)
     long_run, extras = None, None
-    if world == 1 and not args.no_extras:
+    if world == 1 and not args.no_extras and not fp8:
         long_run, t = extra_runs(torch, kv, t, Q, K, V, O)
         extras, t = run_extras(torch, wm, device, kv, t, Q, K, V, O, window,
                                elapsed_ms / args.steps)
@@ -446,10 +465,12 @@ def run_ours(args, world, rank, local):
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(elapsed_ms / args.steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": config_dict(world),
+        "config": config_dict(world, args.kv_format),
         "tflops_per_step": round(step_tflops, 1),
         "frac_of_bf16_peak_step": round(step_tflops / peak, 4),
-        "roofline": {"kernel": "attend_kernel<64> (fused record write)", "bound": "tensor",
+        "roofline": {"kernel": ("per block: quantize_pair_kernel + widen_pair_kernel + attend_kernel<64>"
+                                if fp8 else "attend_kernel<64> (fused record write)"),
+                     "bound": "tensor",
                      "achieved": round(achieved_tflops, 1), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved_tflops / peak, 4),
                      "peak_source": f"{peak_name} ({pk['source']}); timed region "
@@ -460,8 +481,8 @@ def run_ours(args, world, rank, local):
                             f"(run time - evictions) / ({BLOCKS} x {n_rf}) launches",
                      "run_ms": round(rf_total_ms, 3), "evict_ms": round(evict_ms, 3),
                      "share_from_events": round(1.0 - evict_ms / rf_total_ms, 4),
-                     "ncu_share": load_ncu_share(),
-                     "flop_per_launch": ATTN_FLOP, "traffic": load_traffic()},
+                     "ncu_share": None if fp8 else load_ncu_share(),
+                     "flop_per_launch": ATTN_FLOP, "traffic": None if fp8 else load_traffic()},
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clk.summary(),
@@ -990,11 +1011,17 @@ class OracleStepper:
     keys).
     """
 
-    def __init__(self, layout=None, config_id=CONFIG_ID, t_steady=T_STEADY):
+    def __init__(self, layout=None, config_id=CONFIG_ID, t_steady=T_STEADY, kv_format="bf16"):
         from oracle import FrameMemory, Layout
         self.L = layout if layout is not None else Layout(GH, GW, X, Y, W, heads=HEADS, d=D)
         self.config_id = config_id
-        self.mem = FrameMemory(self.L, 1, track_records=False)
+        self.kv_format = kv_format
+        if kv_format == "e4m3":
+            sc = np.full((1, self.L.heads), FP8_SCALE, np.float32)
+            self.mem = FrameMemory(self.L, 1, track_records=False, kv_format="e4m3", k_scale=sc,
+                                   v_scale=sc)
+        else:
+            self.mem = FrameMemory(self.L, 1, track_records=False)
         L = self.L
         for t in range(t_steady):
             self.mem.advance(t)
@@ -1053,7 +1080,7 @@ def gpu_parity_on_stepper(stepper, torch, wm):
     (all heads) within max-abs 2e-2 and relative L2 5e-3.  Raises on a mismatch."""
     from oracle import attend_memory
     L = stepper.L
-    kv = wm.KVMemory(1, L.heads, L.d, L.grid_h, L.grid_w, L.X, L.Y, L.W)
+    kv = make_memory(wm, stepper.kv_format, 1, L.heads, L.d, L.grid_h, L.grid_w, L.X, L.Y, L.W)
 
     def dev(bits):
         return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
@@ -1070,8 +1097,11 @@ def gpu_parity_on_stepper(stepper, torch, wm):
     torch.cuda.synchronize()
     kv.sync_status()
     kd, vd = kv.kv_views(0)
-    kb = kd.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
-    vb = vd.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    if stepper.kv_format == "e4m3":
+        kb, vb = kd.contiguous().cpu().numpy(), vd.contiguous().cpu().numpy()
+    else:
+        kb = kd.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+        vb = vd.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
     ob = o.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
     kv.close()
     # the oracle's memory after the same frame (a copy: the stepper's own
@@ -1094,14 +1124,14 @@ def gpu_parity_on_stepper(stepper, torch, wm):
         raise RuntimeError(f"parity: attention max_abs {max_abs:.3e} rel_l2 {rel:.3e}")
     return {"buffers": "bit-exact", "rows": int(len(rows)), "heads": L.heads,
             "max_abs": round(max_abs, 6), "rel_l2": round(rel, 7), "frame": t,
-            "call": "wm_write_attend"}
+            "call": "wm_write_attend", "kv_format": stepper.kv_format}
 
 
-def cpu_baseline_and_parity(budget_s: float, torch=None, wm=None):
+def cpu_baseline_and_parity(budget_s: float, torch=None, wm=None, kv_format="bf16"):
     """The oracle timed on the host cores (served block, extrapolated to a
     frame-step), one thread and the scaled memory as well; with ``wm`` given,
     the GPU path is first checked against the oracle on the same inputs."""
-    stepper = OracleStepper()
+    stepper = OracleStepper(kv_format=kv_format)
     parity = gpu_parity_on_stepper(stepper, torch, wm) if wm is not None else None
     per_step, rows, t_attn, _ = stepper.step(budget_s)
     out = {"value": round(1.0 / per_step, 6), "unit": UNIT, "cores": _oracle_threads(),
@@ -1146,7 +1176,7 @@ def run_reference(args, world, rank):
     # size each step so the whole run stays within ~2 minutes
     n_steps = args.warmup + args.steps
     budget = max(0.05, min(2.0, 120.0 / max(1, n_steps)))
-    stepper = OracleStepper()
+    stepper = OracleStepper(kv_format=args.kv_format)
     for _ in range(args.warmup):
         stepper.step(budget)
     per = []
@@ -1163,7 +1193,7 @@ def run_reference(args, world, rank):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": config_dict(world),
+            "config": config_dict(world, args.kv_format),
             "extrapolated": True,
             "seconds_spent": round(spent_total, 2),
             "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
@@ -1186,6 +1216,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kv-format", choices=["bf16", "e4m3"], default="bf16",
+                    help="storage of the frame memory: bf16 (the default workload) or FP8 E4M3 codes "
+                         "with one scale per (block, head); e4m3 runs no extras")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the long runs and the secondary measurements (CUDA graphs, four-pass "
                          "frame, copy kernels' HBM throughput, batch of 8, scaled memory vs dense)")
