@@ -421,7 +421,9 @@ def run_ours(args, world, rank, local):
     barrier(world)
     kv.sync_status()
     elapsed_ms = max_over_ranks(start.elapsed_time(stop), world, device)
-    launches = args.steps * (1 + (3 if fp8 else 1) * BLOCKS)
+    # per step: the eviction, then per block one launch (bf16: fused write and
+    # attention) or two (FP8: record store + widening, attention)
+    launches = args.steps * (1 + (2 if fp8 else 1) * BLOCKS)
 
     # ------------------------------------------------ attention launch time (roofline)
     # The same steps again with an event pair around each eviction only: the
@@ -468,7 +470,7 @@ def run_ours(args, world, rank, local):
         "config": config_dict(world, args.kv_format),
         "tflops_per_step": round(step_tflops, 1),
         "frac_of_bf16_peak_step": round(step_tflops / peak, 4),
-        "roofline": {"kernel": ("per block: quantize_pair_kernel + widen_pair_kernel + attend_kernel<64>"
+        "roofline": {"kernel": ("per block: store_widen_pair_kernel + attend_kernel<64>"
                                 if fp8 else "attend_kernel<64> (fused record write)"),
                      "bound": "tensor",
                      "achieved": round(achieved_tflops, 1), "peak": peak, "unit": "TFLOP/s",
@@ -918,14 +920,14 @@ def extra_fp8(torch, wm, Q, K, V, O, steps=50):
     widen_us = (ms8 - ms16) * 1e3
     widen_bytes = 2 * C * HEADS * D * (1 + 2)         # codes read, bf16 written, K and V
     return {"value": round(1e3 / ms, 3), "unit": UNIT, "ms_per_step": round(ms, 4), "steps": steps,
-            "launches_per_step": 1 + 3 * BLOCKS,
+            "launches_per_step": 1 + 2 * BLOCKS,
             "buffer_bytes": 2 * BLOCKS * C * HEADS * D,
             "tflops_per_step": round(BLOCKS * ATTN_FLOP / (ms * 1e-3) / 1e12, 1),
             "widen": {"us": round(widen_us, 2), "bytes": widen_bytes,
                       "GB_per_s": round(widen_bytes / max(widen_us, 1e-3) / 1e3, 1),
                       "how": f"wm_attend_dense_fp8 minus wm_attend_dense over {C} keys x {HEADS} x {D}, "
                              f"{n} calls each, back to back"},
-            "how": "advance + 28 x write_attend on an E4M3 memory (quantise, widen, attend)"}
+            "how": "advance + 28 x write_attend on an E4M3 memory (store and widen, attend)"}
 
 
 def extra_served_dense(torch, wm, device, ms_step, pk, steps=3):

@@ -105,6 +105,54 @@ __global__ void __launch_bounds__(THREADS) widen_pair_kernel(const uint4* __rest
   }
 }
 
+// The record write and the widening of one block's prefix in one pass
+// (wm_write_attend on an FP8 memory).  Units of 8 values over [0, end) rows of
+// K (blockIdx.y = 0) or V (1): units in [slot_lo, slot_hi) come from the
+// caller's bf16 record -- quantised, stored as codes in the slot, and widened
+// from those codes -- the others are widened from the codes in the buffer.
+__global__ void __launch_bounds__(THREADS) store_widen_pair_kernel(
+    const uint4* __restrict__ k_rec, const uint4* __restrict__ v_rec, uint2* __restrict__ k_codes,
+    uint2* __restrict__ v_codes, uint4* __restrict__ k_out, uint4* __restrict__ v_out, int64_t n8,
+    int64_t slot_lo, int64_t slot_hi, int heads, int d, const float* __restrict__ k_scale,
+    const float* __restrict__ v_scale) {
+  pdl_launch_dependents();
+  pdl_wait_prior();
+  const uint4* rec = blockIdx.y ? v_rec : k_rec;
+  uint2* codes = blockIdx.y ? v_codes : k_codes;
+  uint4* out = blockIdx.y ? v_out : k_out;
+  const float* scale = blockIdx.y ? v_scale : k_scale;
+  const int groups_per_head = d / 8;
+  const int64_t stride = int64_t(gridDim.x) * THREADS;
+  for (int64_t g = int64_t(blockIdx.x) * THREADS + threadIdx.x; g < n8; g += stride) {
+    uint2 c;
+    if (g >= slot_lo && g < slot_hi) {
+      const float s = scale[(g / groups_per_head) % heads];
+      const uint4 x = rec[g - slot_lo];
+      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+      uint32_t q[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        uint16_t h[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const uint32_t pair = w[2 * i + j];
+          h[j] = e4m3x2_from_f32(__fdiv_rn(__uint_as_float(pair << 16), s),
+                                 __fdiv_rn(__uint_as_float(pair & 0xFFFF0000u), s));
+        }
+        q[i] = uint32_t(h[0]) | (uint32_t(h[1]) << 16);
+      }
+      c = make_uint2(q[0], q[1]);
+      codes[g] = c;
+    } else {
+      c = codes[g];
+    }
+    out[g] = make_uint4(bf16x2_from_e4m3x2(static_cast<uint16_t>(c.x & 0xFFFFu)),
+                        bf16x2_from_e4m3x2(static_cast<uint16_t>(c.x >> 16)),
+                        bf16x2_from_e4m3x2(static_cast<uint16_t>(c.y & 0xFFFFu)),
+                        bf16x2_from_e4m3x2(static_cast<uint16_t>(c.y >> 16)));
+  }
+}
+
 unsigned grid_for(int64_t units, int sms) {
   int64_t want = (units + THREADS - 1) / THREADS;
   const int64_t cap = int64_t(sms) * 8;
@@ -125,6 +173,23 @@ cudaError_t launch_quantize_pair(const void* k_src, const void* v_src, void* k_d
                     static_cast<const uint4*>(k_src), static_cast<const uint4*>(v_src),
                     static_cast<uint2*>(k_dst), static_cast<uint2*>(v_dst), n8, heads, d, k_scale,
                     v_scale);
+}
+
+cudaError_t launch_store_widen_pair(const void* k_rec, const void* v_rec, void* k_codes, void* v_codes,
+                                    void* k_out, void* v_out, int64_t elems, int64_t slot_lo,
+                                    int64_t slot_hi, int heads, int d, const float* k_scale,
+                                    const float* v_scale, cudaStream_t stream) {
+  if (elems <= 0) return cudaSuccess;
+  if (elems % 8 || slot_lo % 8 || slot_hi % 8 || d % 8 || slot_lo < 0 || slot_hi < slot_lo ||
+      slot_hi > elems)
+    return cudaErrorInvalidValue;
+  const int64_t n8 = elems / 8;
+  dim3 grid(grid_for(n8, device_sm_count()), 2);
+  return launch_pdl(store_widen_pair_kernel, grid, dim3(THREADS), 0, stream,
+                    static_cast<const uint4*>(k_rec), static_cast<const uint4*>(v_rec),
+                    static_cast<uint2*>(k_codes), static_cast<uint2*>(v_codes),
+                    static_cast<uint4*>(k_out), static_cast<uint4*>(v_out), n8, slot_lo / 8,
+                    slot_hi / 8, heads, d, k_scale, v_scale);
 }
 
 cudaError_t launch_widen_pair(const void* k_codes, const void* v_codes, void* k_out, void* v_out,

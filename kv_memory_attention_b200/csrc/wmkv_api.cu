@@ -352,10 +352,20 @@ int wm_write_attend(wm_kvbuf* h, int block, int64_t t, const void* Q, const void
   const int64_t end = end_at(h->HW, h->X, h->Y, h->W, t);
   cudaError_t e;
   if (h->kv_format == WM_KV_E4M3) {
-    // the attention must see the stored (quantised) record: store, then attend
+    // the attention must see the stored (quantised) record: one pass stores
+    // the record's codes in the slot and widens the whole prefix (the record
+    // from its own codes), then the attention reads the widened prefix
     h->written[block] = -1;
-    e = store_record(h, block, row0, K, V, s);
-    if (e == cudaSuccess) e = attend_prefix(h, block, Q, O, s);
+    const int64_t per_row = int64_t(h->heads) * h->d;
+    uint8_t* wk = h->widened;
+    uint8_t* wv = h->widened + h->C * per_row * 2;
+    e = wmkv::launch_store_widen_pair(K, V, kbuf, vbuf, wk, wv, end * per_row, row0 * per_row,
+                                      (row0 + h->R) * per_row, h->heads, h->d,
+                                      block_k_scale(h, block), block_v_scale(h, block), s);
+    const wmkv::KVSegment seg = {wk, wv, end};
+    if (e == cudaSuccess)
+      e = wmkv::launch_attend(Q, O, h->R, &seg, 1, h->heads, h->d, h->status, nullptr, h->wait_limit,
+                              block_k_scale(h, block), block_v_scale(h, block), s);
   } else if (wmkv::attend_copies_in_kernel(h->d)) {
     // keys: buffer rows before the slot, buffer rows after it, and the record
     // itself from the caller (the slot is being written by the same launch)

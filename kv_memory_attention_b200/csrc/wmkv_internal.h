@@ -81,6 +81,14 @@ int device_sm_count();
 cudaError_t launch_quantize_pair(const void* k_src, const void* v_src, void* k_dst, void* v_dst,
                                  int64_t elems, int heads, int d, const float* k_scale,
                                  const float* v_scale, cudaStream_t stream);
+// Both in one pass over `elems` values of K and of V: values [slot_lo,
+// slot_hi) come from the bf16 record (quantised into k_codes/v_codes there),
+// the rest from the codes already stored; all are widened into k_out/v_out.
+// elems, slot_lo and slot_hi are multiples of 8.
+cudaError_t launch_store_widen_pair(const void* k_rec, const void* v_rec, void* k_codes, void* v_codes,
+                                    void* k_out, void* v_out, int64_t elems, int64_t slot_lo,
+                                    int64_t slot_hi, int heads, int d, const float* k_scale,
+                                    const float* v_scale, cudaStream_t stream);
 // Widen `elems` E4M3 codes of K and of V (elems a multiple of 16) to the
 // bfloat16 values they hold (exact).
 cudaError_t launch_widen_pair(const void* k_codes, const void* v_codes, void* k_out, void* v_out,
