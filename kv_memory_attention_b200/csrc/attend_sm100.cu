@@ -12,7 +12,7 @@
 //   warp 9      owns TMEM (512 columns) and issues S_j = Q K_j^T
 //               (tcgen05.mma SS: both operands K-major in smem)
 //   warps 10/11 issue O_g += P_j V_j for even / odd tiles (tcgen05.mma TS: P
-//               from TMEM, V MN-major in smem); three issuing threads keep the
+//               from TMEM, V MN-major in smem); three issuing warps keep the
 //               tensor core fed while each waits on barriers and commits.
 //               For d = 128 warp 9 issues everything, in order.
 //   warps 0-3   softmax warpgroup 0: even key tiles, S0/P0/O0 in TMEM
@@ -279,6 +279,27 @@ __device__ __forceinline__ void issue_pv(uint64_t dv, uint32_t p_tmem, uint32_t 
            (accumulate | uint32_t(kk > 0)));
 }
 
+// Warp-wide forms of the two (the whole warp calls them; one lane issues).
+template <int D>
+__device__ __forceinline__ void issue_s_warp(uint64_t dq, uint64_t dk, uint32_t d_s) {
+  using C = Cfg<D>;
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint64_t off = uint64_t(((kk / 4) * C::SUB_BYTES + (kk % 4) * 32) >> 4);
+    mma_ss_elect(d_s, dq + off, dk + off, C::IDESC_S, kk > 0 ? 1u : 0u);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void issue_pv_warp(uint64_t dv, uint32_t p_tmem, uint32_t d_o,
+                                              uint32_t accumulate) {
+  using C = Cfg<D>;
+#pragma unroll
+  for (int kk = 0; kk < BN / 16; ++kk)
+    mma_ts_elect(d_o, p_tmem + kk * 8, dv + uint64_t((kk * 2048) >> 4), C::IDESC_O,
+                 (accumulate | uint32_t(kk > 0)));
+}
+
 template <int D>
 __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_constant__ AttendParams p) {
   using C = Cfg<D>;
@@ -447,11 +468,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
     // (try_wait) so that the issuers do not take issue slots from the
     // softmax warps on the same SM sub-partitions; waits on TMA data that
     // normally has landed already (K_full, V_full) poll (test_wait).
-    // Two issuing threads share the tensor core: warp 9 issues S = Q K^T,
-    // warp 10 issues O += P V, so that each thread's barrier waits and
-    // commits overlap with the other's MMAs.  A commit tracks only the
-    // committing thread's own MMAs.
-    if (lane == 0) {
+    // Three issuing warps share the tensor core: warp 9 issues S = Q K^T,
+    // warps 10/11 issue O += P V, so that each one's barrier waits and
+    // commits overlap with the others' MMAs.  A commit tracks only the
+    // committing thread's own MMAs.  For d = 64 the issuing warps stay
+    // converged (every lane waits, one elected lane issues: the wait results
+    // are made warp-uniform first); for d = 128 lane 0 alone runs the loop.
+    if (C::TWO_ISSUERS || lane == 0) {
       constexpr uint64_t TILE16 = C::TILE_BYTES >> 4;
       bool ok = true;
       if (!C::TWO_ISSUERS) {
@@ -502,7 +525,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
         const uint64_t dk0 = sdesc_sw128(sbase + C::K_OFF, 16, 1024);
         uint32_t k_st = 0, k_ph = 0;  // ring slot / phase of the next K tile
         uint32_t fr_ph = 0;           // bit g: phase of the barrier that frees S_g
-        ok = mbar_spin_bounded(bar(C::B_Q), 0, abort_flag, p.wait_limit);
+        ok = __all_sync(0xffffffffu, mbar_spin_bounded(bar(C::B_Q), 0, abort_flag, p.wait_limit));
         for (int j = 0; ok && j < nkv; ++j) {
           const int g = j & 1;
           if (j >= 2) {
@@ -510,20 +533,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
             // own columns) or once P_{j-2}.V_{j-2} has completed (d = 128: P
             // overwrote S_{j-2})
             const int fb = C::P_SEP ? C::B_SFREE + g : C::B_ODONE + g;
-            if (!mbar_wait_bounded(bar(fb), (fr_ph >> g) & 1, abort_flag, p.wait_limit)) {
+            if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar(fb), (fr_ph >> g) & 1, abort_flag,
+                                                           p.wait_limit))) {
               ok = false;
               break;
             }
             fr_ph ^= 1u << g;
           }
-          if (!mbar_spin_bounded(bar(C::B_KFULL + k_st), k_ph, abort_flag, p.wait_limit)) {
+          if (!__all_sync(0xffffffffu, mbar_spin_bounded(bar(C::B_KFULL + k_st), k_ph, abort_flag,
+                                                         p.wait_limit))) {
             ok = false;
             break;
           }
           tc_fence_after();
-          issue_s<D>(dq, dk0 + k_st * TILE16, tmem + (g ? C::S_COL1 : C::S_COL0));
-          tc_commit(bar(C::B_SFULL + g));
-          tc_commit(bar(C::B_KEMPTY + k_st));
+          issue_s_warp<D>(dq, dk0 + k_st * TILE16, tmem + (g ? C::S_COL1 : C::S_COL0));
+          tc_commit_elect(bar(C::B_SFULL + g));
+          tc_commit_elect(bar(C::B_KEMPTY + k_st));
           if (++k_st == C::NK) { k_st = 0; k_ph ^= 1; }
         }
       } else {
@@ -537,25 +562,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
         for (int j = g; ok && j < nkv; j += 2) {
           const int v_st = j % C::NV;
           const uint32_t v_ph = (j / C::NV) & 1;
-          if (!mbar_wait_bounded(bar(C::B_PFULL + g), pf_ph, abort_flag, p.wait_limit) ||
-              !mbar_spin_bounded(bar(C::B_VFULL + v_st), v_ph, abort_flag, p.wait_limit)) {
+          if (!__all_sync(0xffffffffu,
+                          mbar_wait_bounded(bar(C::B_PFULL + g), pf_ph, abort_flag, p.wait_limit) &&
+                              mbar_spin_bounded(bar(C::B_VFULL + v_st), v_ph, abort_flag,
+                                                p.wait_limit))) {
             ok = false;
             break;
           }
           pf_ph ^= 1;
           tc_fence_after();
-          issue_pv<D>(dv0 + v_st * TILE16, p_tm, o_tm, j >= 2 ? 1u : 0u);
-          tc_commit(bar(C::B_ODONE + g));
-          tc_commit(bar(C::B_VEMPTY + v_st));
+          issue_pv_warp<D>(dv0 + v_st * TILE16, p_tm, o_tm, j >= 2 ? 1u : 0u);
+          tc_commit_elect(bar(C::B_ODONE + g));
+          tc_commit_elect(bar(C::B_VEMPTY + v_st));
         }
-        if (ok) tc_commit(bar(C::B_OFINAL));
+        if (ok) tc_commit_elect(bar(C::B_OFINAL));
       }
       }
       if (!ok) {
         // let this thread's MMAs finish before TMEM is released
         volatile int no_abort = 0;
         const int db = C::B_DRAIN + (warp - 9);
-        tc_commit(bar(db));
+        if (C::TWO_ISSUERS)
+          tc_commit_elect(bar(db));
+        else
+          tc_commit(bar(db));
         mbar_wait_bounded(bar(db), 0, &no_abort, DRAIN_LIMIT_CYCLES);
       }
     }
