@@ -102,7 +102,8 @@ enum { WM_KV_BF16 = 0, WM_KV_E4M3 = 1 };
  * the dequantised prefix (the codes are widened to bf16 in the handle's
  * scratch, 2 * C * heads * d * 2 bytes allocated here, and the scales enter
  * in float32: K's with the softmax scale, V's with the output
- * normalisation).  wm_write_attend is three launches (store, widen, attend).
+ * normalisation).  wm_write_attend is two launches: one stores the record's
+ * codes in its slot and widens the block's prefix, one attends.
  * Calls on one E4M3 handle must be ordered on the device (one stream, or
  * events between streams): they share its scratch.  wm_set_sink returns
  * WM_ERR_UNSUPPORTED for this format.  Other arguments and errors as for
