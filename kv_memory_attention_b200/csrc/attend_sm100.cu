@@ -468,55 +468,58 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
     // (try_wait) so that the issuers do not take issue slots from the
     // softmax warps on the same SM sub-partitions; waits on TMA data that
     // normally has landed already (K_full, V_full) poll (test_wait).
-    // Three issuing warps share the tensor core: warp 9 issues S = Q K^T,
-    // warps 10/11 issue O += P V, so that each one's barrier waits and
-    // commits overlap with the others' MMAs.  A commit tracks only the
-    // committing thread's own MMAs.  For d = 64 the issuing warps stay
-    // converged (every lane waits, one elected lane issues: the wait results
-    // are made warp-uniform first); for d = 128 lane 0 alone runs the loop.
-    if (C::TWO_ISSUERS || lane == 0) {
+    // For d = 64 three issuing warps share the tensor core: warp 9 issues
+    // S = Q K^T, warps 10/11 issue O += P V, so that each one's barrier waits
+    // and commits overlap with the others' MMAs; for d = 128 warp 9 issues
+    // everything.  A commit tracks only the committing thread's own MMAs.
+    // The issuing warps stay converged: every lane waits, the wait results are
+    // made warp-uniform, and one elected lane issues each MMA and commit.
+    {
       constexpr uint64_t TILE16 = C::TILE_BYTES >> 4;
       bool ok = true;
       if (!C::TWO_ISSUERS) {
-        // d = 128: one thread issues everything in order; S_{j+2} follows
+        // d = 128: one warp issues everything in order; S_{j+2} follows
         // P_j.V_j in the MMA pipe, which is what lets P overwrite S_j in place
         if (warp == 9) {
           const uint64_t dq = sdesc_sw128(sbase + C::Q_OFF, 16, 1024);
           const uint64_t dk0 = sdesc_sw128(sbase + C::K_OFF, 16, 1024);
           const uint64_t dv0 = sdesc_sw128(sbase + C::V_OFF, C::SUB_BYTES, 1024);
           uint32_t k_st = 0, k_ph = 0, v_st = 0, v_ph = 0, pf_ph = 0;
-          ok = mbar_spin_bounded(bar(C::B_Q), 0, abort_flag, p.wait_limit);
+          ok = __all_sync(0xffffffffu, mbar_spin_bounded(bar(C::B_Q), 0, abort_flag, p.wait_limit));
           auto do_s = [&](int g) -> bool {
-            if (!mbar_spin_bounded(bar(C::B_KFULL + k_st), k_ph, abort_flag, p.wait_limit))
+            if (!__all_sync(0xffffffffu, mbar_spin_bounded(bar(C::B_KFULL + k_st), k_ph, abort_flag,
+                                                           p.wait_limit)))
               return false;
             tc_fence_after();
-            issue_s<D>(dq, dk0 + k_st * TILE16, tmem + (g ? C::S_COL1 : C::S_COL0));
-            tc_commit(bar(C::B_SFULL + g));
-            tc_commit(bar(C::B_KEMPTY + k_st));
+            issue_s_warp<D>(dq, dk0 + k_st * TILE16, tmem + (g ? C::S_COL1 : C::S_COL0));
+            tc_commit_elect(bar(C::B_SFULL + g));
+            tc_commit_elect(bar(C::B_KEMPTY + k_st));
             if (++k_st == C::NK) { k_st = 0; k_ph ^= 1; }
             return true;
           };
           for (int j = 0; ok && j < 2 && j < nkv; ++j) ok = do_s(j);
           for (int j = 0; ok && j < nkv; ++j) {
             const int g = j & 1;
-            if (!mbar_wait_bounded(bar(C::B_PFULL + g), (pf_ph >> g) & 1, abort_flag,
-                                   p.wait_limit) ||
-                !mbar_spin_bounded(bar(C::B_VFULL + v_st), v_ph, abort_flag, p.wait_limit)) {
+            if (!__all_sync(0xffffffffu,
+                            mbar_wait_bounded(bar(C::B_PFULL + g), (pf_ph >> g) & 1, abort_flag,
+                                              p.wait_limit) &&
+                                mbar_spin_bounded(bar(C::B_VFULL + v_st), v_ph, abort_flag,
+                                                  p.wait_limit))) {
               ok = false;
               break;
             }
             pf_ph ^= 1u << g;
             tc_fence_after();
-            issue_pv<D>(dv0 + v_st * TILE16, tmem + (g ? C::P_COL1 : C::P_COL0),
-                        tmem + (g ? C::O_COL1 : C::O_COL0), j >= 2 ? 1u : 0u);
-            tc_commit(bar(C::B_ODONE + g));
-            tc_commit(bar(C::B_VEMPTY + v_st));
+            issue_pv_warp<D>(dv0 + v_st * TILE16, tmem + (g ? C::P_COL1 : C::P_COL0),
+                             tmem + (g ? C::O_COL1 : C::O_COL0), j >= 2 ? 1u : 0u);
+            tc_commit_elect(bar(C::B_ODONE + g));
+            tc_commit_elect(bar(C::B_VEMPTY + v_st));
             if (++v_st == C::NV) { v_st = 0; v_ph ^= 1; }
             if (j + 2 < nkv && !(ok = do_s(g))) break;
           }
           if (ok) {
-            tc_commit(bar(C::B_OFINAL));
-            tc_commit(bar(C::B_OFINAL));
+            tc_commit_elect(bar(C::B_OFINAL));
+            tc_commit_elect(bar(C::B_OFINAL));
           }
         }
       } else {
@@ -582,10 +585,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
         // let this thread's MMAs finish before TMEM is released
         volatile int no_abort = 0;
         const int db = C::B_DRAIN + (warp - 9);
-        if (C::TWO_ISSUERS)
-          tc_commit_elect(bar(db));
-        else
-          tc_commit(bar(db));
+        tc_commit_elect(bar(db));
         mbar_wait_bounded(bar(db), 0, &no_abort, DRAIN_LIMIT_CYCLES);
       }
     }
