@@ -112,9 +112,10 @@ struct Cfg {
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;  // 1024-byte alignment slack
   // TMEM columns
   static constexpr bool P_SEP = (D == 64);
-  // d = 64: S and P.V MMAs come from two issuing threads (their MMAs are short,
-  // so per-tile waits and commits would otherwise leave the tensor core idle);
-  // d = 128: one issuer, which keeps S_{j+2} behind P_j.V_j in issue order.
+  // d = 64: S and P.V MMAs come from separate issuing warps (their MMAs are
+  // short, so per-tile waits and commits would otherwise leave the tensor core
+  // idle); d = 128: one issuing warp, which keeps S_{j+2} behind P_j.V_j in
+  // issue order.
   static constexpr bool TWO_ISSUERS = P_SEP;
   static constexpr uint32_t S_COL0 = 0, S_COL1 = 128;
   static constexpr uint32_t P_COL0 = P_SEP ? 256 : S_COL0;
@@ -257,29 +258,10 @@ __device__ __forceinline__ void record_timeout(int* status) {
   if (status) atomicExch(status, DEV_TIMEOUT);
 }
 
-// MMA issue helpers.  Descriptors are built once; the start-address field
-// (bits 0-13, in 16-byte units) is advanced by compile-time offsets, so the
-// issuing thread spends its cycles on tcgen05.mma and not on descriptor math.
-template <int D>
-__device__ __forceinline__ void issue_s(uint64_t dq, uint64_t dk, uint32_t d_s) {
-  using C = Cfg<D>;
-#pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    const uint64_t off = uint64_t(((kk / 4) * C::SUB_BYTES + (kk % 4) * 32) >> 4);
-    mma_ss(d_s, dq + off, dk + off, C::IDESC_S, kk > 0 ? 1u : 0u);
-  }
-}
-
-template <int D>
-__device__ __forceinline__ void issue_pv(uint64_t dv, uint32_t p_tmem, uint32_t d_o, uint32_t accumulate) {
-  using C = Cfg<D>;
-#pragma unroll
-  for (int kk = 0; kk < BN / 16; ++kk)
-    mma_ts(d_o, p_tmem + kk * 8, dv + uint64_t((kk * 2048) >> 4), C::IDESC_O,
-           (accumulate | uint32_t(kk > 0)));
-}
-
-// Warp-wide forms of the two (the whole warp calls them; one lane issues).
+// MMA issue helpers, called by a whole converged warp (one elected lane
+// issues).  Descriptors are built once; the start-address field (bits 0-13,
+// in 16-byte units) is advanced by compile-time offsets, so the issuing warp
+// spends its cycles on tcgen05.mma and not on descriptor math.
 template <int D>
 __device__ __forceinline__ void issue_s_warp(uint64_t dq, uint64_t dk, uint32_t d_s) {
   using C = Cfg<D>;
@@ -464,14 +446,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
     }
   } else if (warp >= 9) {
     // ------------------------------------------------------------ MMA issuers
-    // Waits on the softmax warpgroups (S_free, P_full) suspend the thread
-    // (try_wait) so that the issuers do not take issue slots from the
+    // Waits on the softmax warpgroups (S_free, P_full) suspend the waiting
+    // lanes (try_wait) so that the issuers do not take issue slots from the
     // softmax warps on the same SM sub-partitions; waits on TMA data that
     // normally has landed already (K_full, V_full) poll (test_wait).
     // For d = 64 three issuing warps share the tensor core: warp 9 issues
     // S = Q K^T, warps 10/11 issue O += P V, so that each one's barrier waits
     // and commits overlap with the others' MMAs; for d = 128 warp 9 issues
-    // everything.  A commit tracks only the committing thread's own MMAs.
+    // everything.  A commit tracks only the MMAs its own lane issued.
     // The issuing warps stay converged: every lane waits, the wait results are
     // made warp-uniform, and one elected lane issues each MMA and commit.
     {
@@ -555,7 +537,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
           if (++k_st == C::NK) { k_st = 0; k_ph ^= 1; }
         }
       } else {
-        // warp 10: P.V of even tiles, warp 11: odd tiles (each issuing thread
+        // warp 10: P.V of even tiles, warp 11: odd tiles (each issuing warp
         // keeps its own V slots: the V ring has an even number of stages)
         const int g = warp - 10;
         const uint64_t dv0 = sdesc_sw128(sbase + C::V_OFF, C::SUB_BYTES, 1024);
@@ -582,7 +564,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
       }
       }
       if (!ok) {
-        // let this thread's MMAs finish before TMEM is released
+        // let this warp's MMAs finish before TMEM is released
         volatile int no_abort = 0;
         const int db = C::B_DRAIN + (warp - 9);
         tc_commit_elect(bar(db));

@@ -78,8 +78,9 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
   }
 }
 
-// Non-suspending probe of a phase (used by the single MMA-issuing threads:
-// right after tcgen05.commit a test_wait returns sooner than a try_wait).
+// Non-suspending probe of a phase (used by the MMA-issuing warps for data
+// that normally has landed already: there a test_wait returns sooner than a
+// try_wait).
 __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
