@@ -1210,6 +1210,35 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def run_dense_case(spec: str, calls: int):
+    """``LQ,LK,HEADS,D``: ``calls`` back-to-back dense attention calls of that
+    shape on synthetic N(0,1) bf16 inputs, timed with CUDA events (a small,
+    fixed case for kernel captures: one launch per call).  Prints one line."""
+    import torch
+    import kv_memory_attention_b200 as wm
+    lq, lk, heads, d = (int(x) for x in spec.split(","))
+    g = torch.Generator(device="cuda").manual_seed(11)
+    q, k, v = (torch.randn(n, heads, d, device="cuda", dtype=torch.bfloat16, generator=g)
+               for n in (lq, lk, lk))
+    o = torch.empty(lq, heads, d, device="cuda", dtype=torch.bfloat16)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for _ in range(3):
+        wm.wm_attend_dense(q, k, v, o, lq, lk, heads, d, status)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(calls):
+        wm.wm_attend_dense(q, k, v, o, lq, lk, heads, d, status)
+    e1.record()
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, "a bounded wait ran out"
+    us = e0.elapsed_time(e1) * 1e3 / calls
+    flop = 4.0 * lq * lk * heads * d
+    print(json.dumps({"dense": {"lq": lq, "lk": lk, "heads": heads, "d": d, "calls": calls,
+                                "us_per_call": round(us, 2), "tflops": round(flop / us / 1e6, 1)}}),
+          flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -1227,7 +1256,13 @@ def main():
     ap.add_argument("--ncu-csv", help="summarise this ncu --csv capture and exit (no GPU)")
     ap.add_argument("--ncu-out", help="JSON file the summary is written to")
     ap.add_argument("--ncu-cmd", default="", help="the ncu command line, recorded in the summary")
+    ap.add_argument("--dense", metavar="LQ,LK,HEADS,D",
+                    help="time only dense attention calls of this shape (a fixed case for kernel "
+                         "captures; --steps calls) and exit")
     args = ap.parse_args()
+    if args.dense:
+        run_dense_case(args.dense, args.steps)
+        return
     if args.ncu_csv:
         summary = summarize_ncu_csv(args.ncu_csv, args.ncu_cmd)
         with open(args.ncu_out, "w") as f:
