@@ -229,12 +229,12 @@ def _profile_entry(path: str, prefix: str, files=ATTEND_SOURCES):
 def load_traffic():
     """DRAM bytes (read + write) per attention launch from the committed ncu JSON,
     or None when the kernel sources changed since it was captured."""
-    k = _profile_entry(TRAFFIC_JSON, "attend_kernel<64>")
+    k = _profile_entry(TRAFFIC_JSON, "attend_kernel<64")
     return None if k is None else k.get("dram_bytes_per_launch")
 
 
 def load_ncu_share():
-    k = _profile_entry(LAUNCHES_JSON, "attend_kernel<64>")
+    k = _profile_entry(LAUNCHES_JSON, "attend_kernel<64")
     return None if k is None else k.get("share")
 
 

@@ -79,6 +79,10 @@ enum {
  * record" (R = grid_h*grid_w raw rows followed by X summary rows).
  * Buffers are zero-filled, in one allocation of
  * blocks * 2 * C * heads * d * 2 bytes (block b's K buffer first, then its V).
+ * The handle also holds a scratch of (SM count) * 128 * (d + 2) floats: an
+ * attention launch of more than one wave of (query tile, head) CTAs whose
+ * last wave is at most half full splits that wave's query tiles by key range
+ * and merges the partial results in a second launch.
  * Requirements: blocks >= 1, heads >= 1, d in {64, 128}, grid_h >= 1,
  * grid_w >= 1, X >= 1, 0 <= Y <= W (W == Y gives an empty SUM region).
  * Returns WM_ERR_INVALID_ARG / WM_ERR_UNSUPPORTED before touching the device,

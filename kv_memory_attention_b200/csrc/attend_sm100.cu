@@ -233,6 +233,17 @@ struct AttendParams {
   uint4* copy_dst[2];
   int64_t copy_n16;
   uint64_t wait_limit;  // SM cycles per bounded wait
+  // Work of a CTA (linear id c = blockIdx.y * gridDim.x + blockIdx.x): CTAs
+  // c < full_ctas own query tile c mod q_tiles of head c / q_tiles over all
+  // keys; the others split the keys of the remaining query tiles, split_chunks
+  // CTAs per tile, chunk_tiles key tiles each, and leave unnormalised partial
+  // results in `part` (BM x D fp32 O, then BM row maxima and BM row sums per
+  // CTA) for the combine launch.
+  int q_tiles;
+  int64_t full_ctas;
+  int split_chunks;
+  int chunk_tiles;
+  float* part;
   // per-head factors of the stored keys and values (FP8 buffers), or null
   const float* k_scale;
   const float* v_scale;
@@ -282,7 +293,10 @@ __device__ __forceinline__ void issue_pv_warp(uint64_t dv, uint32_t p_tmem, uint
                  (accumulate | uint32_t(kk > 0)));
 }
 
-template <int D>
+// SPLIT: the launch splits its last wave's query tiles by key range (see
+// AttendParams); a launch without a split uses the instantiation that has no
+// trace of it.
+template <int D, bool SPLIT>
 __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_constant__ AttendParams p) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -297,9 +311,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const int q_tile = blockIdx.x;
-  const int head = blockIdx.y;
-  const int nkv = p.seg_tiles_end[p.nseg - 1];
+  // this CTA's (query tile, head) and key tiles [j0, j0 + nkv)
+  const int nkv_all = p.seg_tiles_end[p.nseg - 1];
+  int64_t cta = 0;
+  bool split = false;
+  int q_tile, head, j0 = 0, nkv = nkv_all;
+  if constexpr (SPLIT) {
+    cta = int64_t(blockIdx.y) * gridDim.x + blockIdx.x;
+    split = cta >= p.full_ctas;
+    const int64_t item = split ? p.full_ctas + (cta - p.full_ctas) / p.split_chunks : cta;
+    q_tile = static_cast<int>(item % p.q_tiles);
+    head = static_cast<int>(item / p.q_tiles);
+    if (split) {
+      j0 = static_cast<int>((cta - p.full_ctas) % p.split_chunks) * p.chunk_tiles;
+      nkv = p.chunk_tiles < nkv_all - j0 ? p.chunk_tiles : nkv_all - j0;
+    }
+  } else {
+    q_tile = blockIdx.x;
+    head = blockIdx.y;
+  }
 
   pdl_launch_dependents();
   if (threadIdx.x == 0) {
@@ -409,7 +439,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
           if (i >= C::NK && !mbar_wait_bounded(bar(C::B_KEMPTY + st), ((i / C::NK) - 1) & 1,
                                                abort_flag, p.wait_limit))
             break;
-          const TileLoc tl = tile_loc(p, i);
+          const TileLoc tl = tile_loc(p, j0 + i);
           mbar_expect_tx(bar(C::B_KFULL + st), C::TILE_BYTES);
           for (int s = 0; s < C::SUB; ++s)
             tma_load_3d(sbase + C::K_OFF + st * C::TILE_BYTES + s * C::SUB_BYTES, &p.tm_k[tl.seg],
@@ -422,7 +452,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
           if (jv >= C::NV && !mbar_wait_bounded(bar(C::B_VEMPTY + st), ((jv / C::NV) - 1) & 1,
                                                 abort_flag, p.wait_limit))
             break;
-          const TileLoc tl = tile_loc(p, jv);
+          const TileLoc tl = tile_loc(p, j0 + jv);
           mbar_expect_tx(bar(C::B_VFULL + st), C::TILE_BYTES);
           for (int s = 0; s < C::SUB; ++s)
             tma_load_3d(sbase + C::V_OFF + st * C::TILE_BYTES + s * C::SUB_BYTES, &p.tm_v[tl.seg],
@@ -606,7 +636,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
 #pragma unroll
       for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
       {
-        const int valid = tile_loc(p, j).valid;
+        const int valid = tile_loc(p, j0 + j).valid;
         if (valid < BN) {
 #pragma unroll
           for (int c = 0; c < 128; ++c)
@@ -671,7 +701,42 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
     xch_m[wg * BM + row] = m_ref;
     xch_l[wg * BM + row] = l_run;
     named_bar_sync(1, 256);
-    if (ok && !*abort_flag) {
+    if (ok && !*abort_flag && split) {
+      // unnormalised partial result of this key range: O = O_0 a_0 + O_1 a_1
+      // with the row's reference mf, and l = l_0 a_0 + l_1 a_1
+      const float m0 = xch_m[row], m1 = xch_m[BM + row];
+      const float l0 = xch_l[row], l1 = xch_l[BM + row];
+      const float mf = fmaxf(m0, m1);
+      const float a0 = ex2_approx(m0 - mf);
+      const float a1 = nkv > 1 ? ex2_approx(m1 - mf) : 0.f;
+      const bool has1 = nkv > 1;
+      float* part = p.part + (cta - p.full_ctas) * int64_t(BM * (D + 2));
+      const uint32_t o0 = tmem + lane_off + C::O_COL0;
+      const uint32_t o1 = tmem + lane_off + C::O_COL1;
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        const int col = wg * (D / 2) + c * 32;
+        uint32_t r0[32], r1[32];
+        tmem_ld32(o0 + col, r0);
+        if (has1) tmem_ld32(o1 + col, r1);
+        tmem_wait_ld();
+        float4* dst = reinterpret_cast<float4*>(part + row * D + col);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float x[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            x[k] = __uint_as_float(r0[4 * i + k]) * a0;
+            if (has1) x[k] = fmaf(__uint_as_float(r1[4 * i + k]), a1, x[k]);
+          }
+          dst[i] = make_float4(x[0], x[1], x[2], x[3]);
+        }
+      }
+      if (wg == 0) {
+        part[BM * D + row] = mf;
+        part[BM * D + BM + row] = l0 * a0 + l1 * a1;
+      }
+    } else if (ok && !*abort_flag) {
       const float m0 = xch_m[row], m1 = xch_m[BM + row];
       const float l0 = xch_l[row], l1 = xch_l[BM + row];
       const float mf = fmaxf(m0, m1);
@@ -722,6 +787,54 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
   }
 }
 
+// Merge of a split query tile's partial results: per row, M = max_k m_k and
+//   O = v_scale * sum_k 2^(m_k - M) O_k / sum_k 2^(m_k - M) l_k,
+// rounded to bf16.  One thread per (row, group of 8 columns): blockIdx.x is
+// the split tile (item full_ctas + blockIdx.x), blockIdx.y a slice of rows.
+constexpr int COMBINE_THREADS = 256;
+template <int D>
+__global__ void __launch_bounds__(COMBINE_THREADS) combine_kernel(const float* __restrict__ part,
+                                                                  int64_t full_ctas, int q_tiles,
+                                                                  int split_chunks, int64_t lq,
+                                                                  int heads,
+                                                                  const float* __restrict__ v_scale,
+                                                                  __nv_bfloat16* __restrict__ o) {
+  pdl_launch_dependents();
+  pdl_wait_prior();
+  constexpr int CG = D / 8;
+  constexpr int64_t PART = int64_t(BM) * (D + 2);
+  const int idx = blockIdx.y * COMBINE_THREADS + threadIdx.x;
+  const int row = idx / CG, cg = idx % CG;
+  const int64_t item = full_ctas + blockIdx.x;
+  const int q_tile = static_cast<int>(item % q_tiles);
+  const int head = static_cast<int>(item / q_tiles);
+  const int64_t qrow = int64_t(q_tile) * BM + row;
+  if (row >= BM || qrow >= lq) return;
+  const float* base = part + int64_t(blockIdx.x) * split_chunks * PART;
+  float m = -INFINITY;
+#pragma unroll 4
+  for (int k = 0; k < split_chunks; ++k) m = fmaxf(m, base[k * PART + BM * D + row]);
+  float l = 0.f, acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+  for (int k = 0; k < split_chunks; ++k) {
+    const float* ps = base + k * PART;
+    const float w = exp2f(ps[BM * D + row] - m);
+    l = fmaf(w, ps[BM * D + BM + row], l);
+    const float4 a = reinterpret_cast<const float4*>(ps + row * D + cg * 8)[0];
+    const float4 b = reinterpret_cast<const float4*>(ps + row * D + cg * 8)[1];
+    acc[0] = fmaf(w, a.x, acc[0]); acc[1] = fmaf(w, a.y, acc[1]);
+    acc[2] = fmaf(w, a.z, acc[2]); acc[3] = fmaf(w, a.w, acc[3]);
+    acc[4] = fmaf(w, b.x, acc[4]); acc[5] = fmaf(w, b.y, acc[5]);
+    acc[6] = fmaf(w, b.z, acc[6]); acc[7] = fmaf(w, b.w, acc[7]);
+  }
+  const float sc = (v_scale ? v_scale[head] : 1.f) / l;
+  uint32_t pk[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) pk[i] = pack_bf16x2(acc[2 * i] * sc, acc[2 * i + 1] * sc);
+  *reinterpret_cast<uint4*>(o + (qrow * heads + head) * D + cg * 8) =
+      make_uint4(pk[0], pk[1], pk[2], pk[3]);
+}
+
 // ---------------------------------------------------------------- host side
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
@@ -754,28 +867,43 @@ bool encode_rows_map(CUtensorMap* m, const void* base, int64_t rows, int heads, 
 
 constexpr int MAX_DEVICES = 64;
 
+// Kernel attributes belong to a device: they are set once on each device used,
+// for each instantiation.  setmaxnreg.inc waits until registers are free, so
+// the launch must carry exactly the budget the register split assumes, or the
+// kernel is not launched.
 template <int D>
-cudaError_t launch_d(const AttendParams& prm, int64_t lq, int heads, cudaStream_t stream) {
+cudaError_t launch_d(const AttendParams& prm, dim3 grid, cudaStream_t stream) {
   using C = Cfg<D>;
-  // kernel attributes belong to a device: set them once on each device used
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES)
     return cudaErrorInvalidDevice;
-  static std::once_flag once[MAX_DEVICES];
-  static cudaError_t attr_err[MAX_DEVICES];
-  std::call_once(once[dev], [dev] {
-    cudaError_t e = cudaFuncSetAttribute(attend_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM_ALLOC);
-    // setmaxnreg.inc waits until registers are free: the launch must carry
-    // exactly the budget the split assumes, or the kernel is not launched.
-    cudaFuncAttributes fa;
-    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, attend_kernel<D>);
-    if (e == cudaSuccess && fa.numRegs != LAUNCH_REGS) e = cudaErrorInvalidConfiguration;
-    attr_err[dev] = e;
-  });
-  if (attr_err[dev] != cudaSuccess) return attr_err[dev];
-  dim3 grid(static_cast<unsigned>((lq + BM - 1) / BM), static_cast<unsigned>(heads));
-  return launch_pdl(attend_kernel<D>, grid, dim3(NUM_THREADS), C::SMEM_ALLOC, stream, prm);
+  const int64_t split_tiles = (int64_t(grid.x) * grid.y - prm.full_ctas) / prm.split_chunks;
+  const bool split = split_tiles > 0;
+  static std::once_flag once[2][MAX_DEVICES];
+  static cudaError_t attr_err[2][MAX_DEVICES];
+  auto prepare = [dev](auto kernel, int which) {
+    std::call_once(once[which][dev], [kernel, which, dev] {
+      cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           C::SMEM_ALLOC);
+      cudaFuncAttributes fa;
+      if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, kernel);
+      if (e == cudaSuccess && fa.numRegs != LAUNCH_REGS) e = cudaErrorInvalidConfiguration;
+      attr_err[which][dev] = e;
+    });
+    return attr_err[which][dev];
+  };
+  cudaError_t e = split ? prepare(attend_kernel<D, true>, 1) : prepare(attend_kernel<D, false>, 0);
+  if (e != cudaSuccess) return e;
+  e = split ? launch_pdl(attend_kernel<D, true>, grid, dim3(NUM_THREADS), C::SMEM_ALLOC, stream, prm)
+            : launch_pdl(attend_kernel<D, false>, grid, dim3(NUM_THREADS), C::SMEM_ALLOC, stream, prm);
+  if (e == cudaSuccess && split)
+    e = launch_pdl(combine_kernel<D>,
+                   dim3(static_cast<unsigned>(split_tiles),
+                        static_cast<unsigned>((BM * (D / 8) + COMBINE_THREADS - 1) / COMBINE_THREADS)),
+                   dim3(COMBINE_THREADS), 0, stream,
+                   static_cast<const float*>(prm.part), prm.full_ctas, prm.q_tiles, prm.split_chunks,
+                   prm.lq, prm.heads, prm.v_scale, prm.o);
+  return e;
 }
 
 }  // namespace
@@ -785,7 +913,7 @@ bool attend_copies_in_kernel(int d) { return Cfg<64>::COPY_IN_KERNEL && d == 64;
 cudaError_t launch_attend(const void* q, void* o, int64_t lq, const KVSegment* segs, int nseg,
                           int heads, int d, int* status, const RecordCopy* copy,
                           unsigned long long wait_limit, const float* k_scale,
-                          const float* v_scale, cudaStream_t stream) {
+                          const float* v_scale, float* part, int part_ctas, cudaStream_t stream) {
   if (nseg < 1 || nseg > MAX_SEGS) return cudaErrorInvalidValue;
   AttendParams prm = {};
   if (!encode_rows_map(&prm.tm_q, q, lq, heads, d)) return cudaErrorInvalidValue;
@@ -816,8 +944,36 @@ cudaError_t launch_attend(const void* q, void* o, int64_t lq, const KVSegment* s
     prm.copy_dst[1] = static_cast<uint4*>(copy->v_dst);
     prm.copy_n16 = copy->n16;
   }
-  if (d == 64) return launch_d<64>(prm, lq, heads, stream);
-  if (d == 128) return launch_d<128>(prm, lq, heads, stream);
+  // One CTA per (query tile, head); when that is one or more full waves of the
+  // SMs plus a remainder of at most half a wave, the remainder's query tiles
+  // are split by key range over the SMs the last wave would leave idle (their
+  // partial results merged by the combine launch).
+  const int64_t q_tiles = (lq + BM - 1) / BM;
+  const int64_t items = q_tiles * heads;
+  prm.q_tiles = static_cast<int>(q_tiles);
+  prm.full_ctas = items;
+  prm.split_chunks = 1;
+  prm.chunk_tiles = tiles;
+  prm.part = part;
+  dim3 grid(static_cast<unsigned>(q_tiles), static_cast<unsigned>(heads));
+  const int sms = device_sm_count();
+  if (part && items > sms && items <= 0x7FFFFFFF) {
+    const int64_t tail = items % sms;
+    int chunks = (tail > 0 && tail <= sms / 2) ? static_cast<int>(sms / tail) : 0;
+    if (chunks > tiles) chunks = tiles;
+    if (chunks >= 2) {
+      const int per = (tiles + chunks - 1) / chunks;
+      chunks = (tiles + per - 1) / per;  // every chunk non-empty
+      if (chunks >= 2 && tail * chunks <= part_ctas) {
+        prm.full_ctas = items - tail;
+        prm.split_chunks = chunks;
+        prm.chunk_tiles = per;
+        grid = dim3(static_cast<unsigned>(prm.full_ctas + tail * chunks), 1);
+      }
+    }
+  }
+  if (d == 64) return launch_d<64>(prm, grid, stream);
+  if (d == 128) return launch_d<128>(prm, grid, stream);
   return cudaErrorInvalidValue;
 }
 

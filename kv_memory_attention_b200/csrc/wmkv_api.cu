@@ -44,6 +44,10 @@ struct wm_kvbuf {
   int gap_trigger = 5, gap_target = 1;
   int64_t z0_pos = 0;          // temporal position of the start image
   unsigned long long wait_limit = wmkv::DEFAULT_WAIT_LIMIT_CYCLES;  // attention launches
+  // scratch for attention launches that split their last wave's query tiles
+  // by key range: part_ctas x 128 x (d + 2) floats (part_ctas = SM count)
+  float* part = nullptr;
+  int part_ctas = 0;
 };
 
 namespace {
@@ -153,6 +157,7 @@ static int kvbuf_create(wm_kvbuf** out, int blocks, int heads, int d, int grid_h
     cudaFree(h->status);
     cudaFree(h->scales);
     cudaFree(h->widened);
+    cudaFree(h->part);
     delete h;
     if (e == cudaErrorMemoryAllocation) {
       cudaGetLastError();
@@ -165,6 +170,9 @@ static int kvbuf_create(wm_kvbuf** out, int blocks, int heads, int d, int grid_h
   const size_t total = size_t(h->block_bytes) * size_t(blocks);
   e = cudaMalloc(&h->buf, total);
   if (e == cudaSuccess) e = cudaMalloc(&h->status, sizeof(int));
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&h->part_ctas, cudaDevAttrMultiProcessorCount, h->device);
+  if (e == cudaSuccess)
+    e = cudaMalloc(&h->part, size_t(h->part_ctas) * 128 * (d + 2) * sizeof(float));
   if (e == cudaSuccess && kv_format == WM_KV_E4M3) {
     const size_t ns = size_t(blocks) * heads;
     e = cudaMalloc(&h->scales, 2 * ns * sizeof(float));
@@ -203,6 +211,7 @@ int wm_kvbuf_destroy(wm_kvbuf* h) {
   cudaFree(h->status);
   cudaFree(h->scales);
   cudaFree(h->widened);
+  cudaFree(h->part);
   cudaSetDevice(dev);
   delete h;
   return e == cudaSuccess ? WM_OK : cuda_fail(e);
@@ -302,11 +311,12 @@ static cudaError_t attend_prefix(wm_kvbuf* h, int block, const void* Q, void* O,
     if (e != cudaSuccess) return e;
     const wmkv::KVSegment seg = {wk, wv, end};
     return wmkv::launch_attend(Q, O, h->R, &seg, 1, h->heads, h->d, h->status, nullptr, h->wait_limit,
-                               block_k_scale(h, block), block_v_scale(h, block), s);
+                               block_k_scale(h, block), block_v_scale(h, block), h->part,
+                               h->part_ctas, s);
   }
   const wmkv::KVSegment seg = {kbuf, vbuf, end};
   return wmkv::launch_attend(Q, O, h->R, &seg, 1, h->heads, h->d, h->status, nullptr, h->wait_limit,
-                             nullptr, nullptr, s);
+                             nullptr, nullptr, h->part, h->part_ctas, s);
 }
 
 int wm_write_record(wm_kvbuf* h, int block, int64_t t, const void* K, const void* V,
@@ -365,7 +375,8 @@ int wm_write_attend(wm_kvbuf* h, int block, int64_t t, const void* Q, const void
     const wmkv::KVSegment seg = {wk, wv, end};
     if (e == cudaSuccess)
       e = wmkv::launch_attend(Q, O, h->R, &seg, 1, h->heads, h->d, h->status, nullptr, h->wait_limit,
-                              block_k_scale(h, block), block_v_scale(h, block), s);
+                              block_k_scale(h, block), block_v_scale(h, block), h->part,
+                              h->part_ctas, s);
   } else if (wmkv::attend_copies_in_kernel(h->d)) {
     // keys: buffer rows before the slot, buffer rows after it, and the record
     // itself from the caller (the slot is being written by the same launch)
@@ -378,13 +389,13 @@ int wm_write_attend(wm_kvbuf* h, int block, int64_t t, const void* Q, const void
     segs[nseg++] = {K, V, h->R};
     const wmkv::RecordCopy cp = {K, V, kslot, vslot, n16};
     e = wmkv::launch_attend(Q, O, h->R, segs, nseg, h->heads, h->d, h->status, &cp, h->wait_limit,
-                            nullptr, nullptr, s);
+                            nullptr, nullptr, h->part, h->part_ctas, s);
   } else {
     e = wmkv::launch_copy_pair(K, V, kslot, vslot, n16, s);
     const wmkv::KVSegment seg = {kbuf, vbuf, end};
     if (e == cudaSuccess)
       e = wmkv::launch_attend(Q, O, h->R, &seg, 1, h->heads, h->d, h->status, nullptr,
-                              h->wait_limit, nullptr, nullptr, s);
+                              h->wait_limit, nullptr, nullptr, h->part, h->part_ctas, s);
   }
   if (e != cudaSuccess) return cuda_fail(e);
   h->written[block] = t;
@@ -465,7 +476,7 @@ int wm_attend_dense(const void* Q, const void* K, const void* V, void* O, int64_
   if ((Lq + 127) / 128 > 0x7FFFFFFF || heads > 65535) return WM_ERR_INVALID_ARG;
   const wmkv::KVSegment seg = {K, V, Lk};
   cudaError_t e = wmkv::launch_attend(Q, O, Lq, &seg, 1, heads, d, dev_status, nullptr,
-                                      wmkv::DEFAULT_WAIT_LIMIT_CYCLES, nullptr, nullptr,
+                                      wmkv::DEFAULT_WAIT_LIMIT_CYCLES, nullptr, nullptr, nullptr, 0,
                                       reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
   return WM_OK;
@@ -492,7 +503,7 @@ int wm_attend_dense_fp8(const void* Q, const void* K8, const void* V8, const flo
   const wmkv::KVSegment seg = {wk, wv, Lk};
   if (e == cudaSuccess)
     e = wmkv::launch_attend(Q, O, Lq, &seg, 1, heads, d, dev_status, nullptr,
-                            wmkv::DEFAULT_WAIT_LIMIT_CYCLES, k_scale, v_scale, s);
+                            wmkv::DEFAULT_WAIT_LIMIT_CYCLES, k_scale, v_scale, nullptr, 0, s);
   if (e != cudaSuccess) return cuda_fail(e);
   return WM_OK;
 }

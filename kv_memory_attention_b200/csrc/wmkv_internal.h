@@ -62,10 +62,15 @@ constexpr unsigned long long DEFAULT_WAIT_LIMIT_CYCLES = 4000000000ull;
 
 // k_scale / v_scale (device, one float per head, may be null): the keys and
 // values are the stored numbers times their head's scale (FP8 buffers).
+//
+// part (device, part_ctas x 128 x (d + 2) floats, may be null): scratch that
+// lets a launch of more than one wave of CTAs split the query tiles of its
+// last, partial wave by key range (a second, combine launch follows); null
+// keeps one CTA per (query tile, head).
 cudaError_t launch_attend(const void* q, void* o, int64_t lq, const KVSegment* segs, int nseg,
                           int heads, int d, int* status, const RecordCopy* copy,
                           unsigned long long wait_limit, const float* k_scale,
-                          const float* v_scale, cudaStream_t stream);
+                          const float* v_scale, float* part, int part_ctas, cudaStream_t stream);
 bool attend_copies_in_kernel(int d);
 
 // Keeps the CUDA error's text for wm_last_cuda_error; returns WM_ERR_CUDA.

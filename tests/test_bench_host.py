@@ -99,3 +99,15 @@ def test_both_arms_describe_the_same_workload():
     c = bench.config_dict(2)
     assert c["workload"] == bench.WORKLOAD and c["keys"] == bench.C == 6528 and c["queries"] == bench.R
     assert c["passes_per_frame"] == 1
+
+
+def test_kernel_names_with_template_flags():
+    """The attention kernel is instantiated per head dimension and per split
+    mode; ncu prints both template arguments, and the bench's lookups match
+    any instantiation of the head dimension."""
+    import bench
+    name = bench._kernel_short_name(
+        "void wmkv::(anonymous namespace)::attend_kernel<64, false>(wmkv::(anonymous namespace)::AttendParams)")
+    assert name == "attend_kernel<64, false>"
+    assert name.startswith("attend_kernel<64")
+    assert not bench._kernel_short_name("void x::attend_kernel<128, true>(x::P)").startswith("attend_kernel<64")
