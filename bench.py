@@ -563,19 +563,20 @@ def run_e2e(args, torch, wm, kv, t, rank, world, device, Qd, Kd, Vd):
     ms = max_over_ranks(start.elapsed_time(stop), world, device)
     nbytes = R * HEADS * D * 2
     h2d = 3 * BLOCKS * nbytes
-    # the host link alone: the same bytes in one pinned host -> device copy
-    big_h = torch.empty(h2d, dtype=torch.uint8).pin_memory()
-    big_d = torch.empty(h2d, dtype=torch.uint8, device=device)
-    big_d.copy_(big_h, non_blocking=True)
-    l0, l1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    l0.record()
+    # the host link alone: the step's own input copies (the same pinned buffers,
+    # the same stream), with no kernels running; the fastest of 5 passes
+    link_ms = []
     for _ in range(5):
-        big_d.copy_(big_h, non_blocking=True)
-    l1.record()
-    torch.cuda.synchronize()
-    link_gbs = 5 * h2d / (l0.elapsed_time(l1) * 1e-3) / 1e9
-    del big_h, big_d
+        l0, l1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        l0.record(s_in)
+        with torch.cuda.stream(s_in):
+            for b in range(BLOCKS):
+                dqkv[b].copy_(hqkv[b], non_blocking=True)
+        l1.record(s_in)
+        torch.cuda.synchronize()
+        link_ms.append(l0.elapsed_time(l1))
+    link_gbs = h2d / (min(link_ms) * 1e-3) / 1e9
     return {"value": round(world * args.steps / (ms / 1e3), 3), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": BLOCKS * nbytes,
             "ms_per_step": round(ms / args.steps, 4),
@@ -583,7 +584,7 @@ def run_e2e(args, torch, wm, kv, t, rank, world, device, Qd, Kd, Vd):
             "h2d_bound_ms_per_step": round(h2d / (link_gbs * 1e9) * 1e3, 4),
             "how": "pinned host Q/K/V (one buffer per block) copied in on a copy stream, O copied "
                    "out on another, overlapped with the kernels block by block; the link figure is "
-                   "one pinned copy of the same bytes", "_t": t}
+                   "the fastest of 5 passes of the same input copies with no kernels running", "_t": t}
 
 
 # ---------------------------------------------------------------- secondary measurements
