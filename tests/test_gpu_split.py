@@ -8,7 +8,8 @@ launch merges the partial results.  On a 148-SM B200 these geometries make
 the last 12 and 6 (query tile, head) pairs -- the last query tiles of the
 last head -- are split.  Rows of those tiles and of unsplit ones are checked
 against the oracle through the fused and the separate calls, over frames
-with one to three key segments.
+with one to three key segments, on a bf16 memory and on an FP8 (E4M3) one
+(whose V scale the combine launch applies).
 """
 import numpy as np
 import pytest
@@ -63,5 +64,38 @@ def test_split_last_wave_matches_oracle(wm, L):
         assert_attn_close(ob[rows], attend_memory(mem, 0, q, rows=rows), f"t={t} (end {L.end(t)})")
     kd, vd = kv.kv_views(0)
     assert np.array_equal(host_bits(kd), mem.K[0]) and np.array_equal(host_bits(vd), mem.V[0])
+    kv.sync_status()
+    kv.close()
+
+
+@pytest.mark.parametrize("L", CASES, ids=lambda L: f"d{L.d}-h{L.heads}-R{L.R}")
+def test_split_last_wave_fp8_memory(wm, L):
+    # scales that are not powers of two, one per head, for K and for V
+    rng = np.random.default_rng(83)
+    ks = rng.uniform(1 / 150, 1 / 40, size=(1, L.heads)).astype(np.float32)
+    vs = rng.uniform(1 / 150, 1 / 40, size=(1, L.heads)).astype(np.float32)
+    kv = wm.KVMemory(1, L.heads, L.d, L.grid_h, L.grid_w, L.X, L.Y, L.W, kv_format="e4m3",
+                     k_scale=ks.ravel(), v_scale=vs.ravel())
+    mem = FrameMemory(L, 1, kv_format="e4m3", k_scale=ks, v_scale=vs)
+    rows = rows_to_check(L)
+    for t in range(3):
+        kv.advance(t)
+        mem.advance(t)
+        q, k, v = si.record_inputs(84, 0, 0, t, 0, L.R, L.heads, L.d)
+        o = torch.full((L.R, L.heads, L.d), float("nan"), dtype=torch.bfloat16, device="cuda")
+        if t % 2 == 0:
+            kv.write_attend(0, t, dev(q), dev(k), dev(v), o)
+        else:
+            kv.write_record(0, t, dev(k), dev(v))
+            kv.attend(0, dev(q), o)
+        mem.write_record(0, t, k, v)
+        torch.cuda.synchronize()
+        ob = host_bits(o)
+        nan = ((ob & 0x7F80) == 0x7F80) & ((ob & 0x007F) != 0)
+        assert not nan.any(), f"t={t}: {int(nan.sum())} output values were never written"
+        assert_attn_close(ob[rows], attend_memory(mem, 0, q, rows=rows), f"t={t} (end {L.end(t)})")
+    kd, vd = kv.kv_views(0)
+    assert np.array_equal(kd.contiguous().cpu().numpy(), mem.K[0])
+    assert np.array_equal(vd.contiguous().cpu().numpy(), mem.V[0])
     kv.sync_status()
     kv.close()
