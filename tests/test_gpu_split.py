@@ -99,3 +99,35 @@ def test_split_last_wave_fp8_memory(wm, L):
     assert np.array_equal(vd.contiguous().cpu().numpy(), mem.V[0])
     kv.sync_status()
     kv.close()
+
+
+def test_split_sessions_on_two_streams(wm):
+    """Two sessions of the split geometry (head dimension 64) driven on two
+    streams with their calls interleaved, so their attention and combine
+    launches may overlap on the device: each handle has its own split scratch."""
+    L = CASES[0]
+    sessions = [(wm.KVMemory(1, L.heads, L.d, L.grid_h, L.grid_w, L.X, L.Y, L.W), FrameMemory(L, 1))
+                for _ in range(2)]
+    streams = [torch.cuda.Stream() for _ in sessions]
+    rows = rows_to_check(L)
+    for t in range(3):
+        ins = [si.record_inputs(85 + s, 0, 0, t, 0, L.R, L.heads, L.d) for s in range(2)]
+        dins = [tuple(dev(x) for x in qkv) for qkv in ins]
+        outs = [torch.full((L.R, L.heads, L.d), float("nan"), dtype=torch.bfloat16, device="cuda")
+                for _ in sessions]
+        torch.cuda.synchronize()
+        for s, (kv, mem) in enumerate(sessions):
+            kv.advance(t, streams[s])
+            mem.advance(t)
+        for s, (kv, mem) in enumerate(sessions):
+            qd, kd, vd = dins[s]
+            kv.write_attend(0, t, qd, kd, vd, outs[s], streams[s])
+            mem.write_record(0, t, ins[s][1], ins[s][2])
+        torch.cuda.synchronize()
+        for s, (kv, mem) in enumerate(sessions):
+            ob = host_bits(outs[s])
+            assert_attn_close(ob[rows], attend_memory(mem, 0, ins[s][0], rows=rows),
+                              f"session {s} t={t}")
+    for kv, _ in sessions:
+        kv.sync_status()
+        kv.close()
