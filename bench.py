@@ -768,7 +768,7 @@ def extra_batch(torch, wm, window, device, sessions=8, steps=20):
                    "each block runs write_attend of every session"}
 
 
-def extra_scaled(torch, wm, device, pk, steps=3):
+def extra_scaled(torch, wm, device, pk, steps=10):
     """The scaled memory (24 heads x 128, 45x80 + X=256, Y=2, W=48: 3856 queries
     x 27,200 keys) at steady state, and the dense full-history baseline it
     replaces (3600 queries x 180,000 keys, wm_attend_dense), 28 blocks each.
