@@ -14,7 +14,8 @@
 //   warps 10/11 issue O_g += P_j V_j for even / odd tiles (tcgen05.mma TS: P
 //               from TMEM, V MN-major in smem); three issuing warps keep the
 //               tensor core fed while each waits on barriers and commits.
-//               For d = 128 warp 9 issues everything, in order.
+//               d = 128 without a redo-flag array: warp 9 issues everything,
+//               in order.
 //   warps 0-3   softmax warpgroup 0: even key tiles, S0/P0/O0 in TMEM
 //   warps 4-7   softmax warpgroup 1: odd key tiles, S1/P1/O1 in TMEM
 // The control warpgroup gives registers back (setmaxnreg) so that each
@@ -31,9 +32,18 @@
 //   of tile j-2 finished: O_g is stable and P_g is free; waiting only now
 //   hides the MMA round trip behind the exponentials) -> rescale O_g if m
 //   moved -> P as bf16 into TMEM -> arrive P_full[g].
-// For d = 128 the TMEM budget (2 S + 2 O of 128 columns) leaves no room for a
-// separate P, so P overwrites the first half of S and S_{j+2} is issued only
-// after P_j.V_j has completed (O_done).
+// d = 128 has two layouts.  Shared O (attention calls of a handle, which
+// owns a per-item flag array): the two warpgroups attend for the same rows,
+// so both P.V issuers accumulate into one O (2 S + 2 P + 1 O of 128, 64,
+// 128 columns), and each row's exponent reference is fixed from the larger
+// of the two warpgroups' first-tile maxima (exchanged once) instead of moved
+// lazily -- S is then released as soon as it is read, as for d = 64.  A tile
+// whose row max exceeds that reference by more than 2^64 (the fp32 headroom
+// of the accumulation) is computed against a clamped reference and its item
+// flagged; a redo launch recomputes flagged items exactly.  Per-warpgroup O
+// (dense calls, no flag array): the TMEM budget (2 S + 2 O of 128 columns)
+// leaves no room for a separate P, so P overwrites the first half of S and
+// S_{j+2} is issued only after P_j.V_j has completed (O_done).
 // The two warpgroups' partial results (m, l, O) are merged row by row at the
 // end and stored as bf16.
 //
@@ -44,6 +54,7 @@
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <mutex>
 
@@ -70,7 +81,7 @@ static_assert(256 * SOFTMAX_REGS + 128 * CONTROL_REGS <= NUM_THREADS * LAUNCH_RE
 // whatever the limit.
 constexpr uint64_t DRAIN_LIMIT_CYCLES = 400000000ull;
 
-template <int D>
+template <int D, bool SHARED = false>
 struct Cfg {
   static constexpr int SUB = D / 64;             // 64-column (128-byte) sub-tiles per row
   static constexpr int SUB_BYTES = BN * 128;     // one sub-tile: 128 rows x 128 B
@@ -78,7 +89,7 @@ struct Cfg {
   // K and V rings.  A K stage is released as soon as its S MMA completes, a
   // V stage after its P.V; the producer keeps K two tiles ahead of V.
   static constexpr int NK = (D == 64) ? 5 : 3;
-  static constexpr int NV = (D == 64) ? 4 : 3;
+  static constexpr int NV = (D == 64) ? 4 : (SHARED ? 2 : 3);
   static constexpr int K_AHEAD = 2;
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + TILE_BYTES;
@@ -89,7 +100,12 @@ struct Cfg {
   static constexpr int COPY_CHUNK_BYTES = 16384;  // per staging buffer (K and V chunk)
   static constexpr int COPY_STAGE_BYTES = COPY_IN_KERNEL ? 2 * COPY_CHUNK_BYTES : 0;
   static constexpr int COPY_OFF = V_OFF + NV * TILE_BYTES;
-  static constexpr int BAR_OFF = COPY_OFF + COPY_STAGE_BYTES;
+  // d = 128: the two warpgroups share one O (they attend for the same rows)
+  // with one exponent reference per row, agreed on once through XCH0
+  static constexpr bool SHARED_O = SHARED;
+  static_assert(!SHARED || D == 128, "the shared O is the head-dimension-128 layout");
+  static constexpr int XCH0_OFF = COPY_OFF + COPY_STAGE_BYTES;  // 2 x BM floats
+  static constexpr int BAR_OFF = XCH0_OFF + (SHARED_O ? 2 * BM * 4 : 0);
   // barrier indices
   static constexpr int B_Q = 0;
   static constexpr int B_KFULL = 1;
@@ -103,7 +119,8 @@ struct Cfg {
   static constexpr int B_OFINAL = B_ODONE + 2;
   static constexpr int B_DRAIN = B_OFINAL + 1;   // 3: one per MMA issuer
   static constexpr int B_COPY = B_DRAIN + 3;     // 2: record copy staging loads (K, V)
-  static constexpr int NBAR = B_COPY + 2;
+  static constexpr int B_OFIRST = B_COPY + 2;    // shared O: the first P.V has completed
+  static constexpr int NBAR = B_OFIRST + (SHARED_O ? 1 : 0);
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;   // [0] tmem base, [1] abort
   // m[2][BM], l[2][BM] for the final merge; they reuse the Q tile, which no
   // MMA reads any more once the last P.V has completed
@@ -111,7 +128,7 @@ struct Cfg {
   static constexpr int SMEM_BYTES = MISC_OFF + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;  // 1024-byte alignment slack
   // TMEM columns
-  static constexpr bool P_SEP = (D == 64);
+  static constexpr bool P_SEP = (D == 64) || SHARED;
   // d = 64: S and P.V MMAs come from separate issuing warps (their MMAs are
   // short, so per-tile waits and commits would otherwise leave the tensor core
   // idle); d = 128: one issuing warp, which keeps S_{j+2} behind P_j.V_j in
@@ -121,12 +138,12 @@ struct Cfg {
   static constexpr uint32_t P_COL0 = P_SEP ? 256 : S_COL0;
   static constexpr uint32_t P_COL1 = P_SEP ? 320 : S_COL1;
   static constexpr uint32_t O_COL0 = P_SEP ? 384 : 256;
-  static constexpr uint32_t O_COL1 = O_COL0 + D;
+  static constexpr uint32_t O_COL1 = SHARED_O ? O_COL0 : O_COL0 + D;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, false, false);
   static constexpr uint32_t IDESC_O = idesc_bf16_f32(BM, D, false, true);
   static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory budget");
-  static_assert(O_COL1 + D <= TMEM_COLS, "TMEM budget");
+  static_assert(O_COL1 + D <= TMEM_COLS && P_COL1 + BM / 2 <= O_COL0, "TMEM budget");
   static_assert(NV % 2 == 0 || !P_SEP, "per-warpgroup P.V issuers need an even V ring");
 };
 
@@ -142,6 +159,10 @@ constexpr int poly_pairs_per_8() {
 // log2 units: O and l are rescaled only when the row max grows by more than
 // 2^8, so every exponential of a tile lies in (0, 2^8].
 constexpr float RESCALE_THRESHOLD = 8.f;
+// shared O (d = 128): a tile whose row max exceeds the fixed reference by more
+// than this many powers of two is flagged (its exponentials would leave the
+// fp32 headroom of the accumulation)
+constexpr float SHARED_REF_HEADROOM = 64.f;
 
 // Largest of the 128 scores of a row: eight independent chains of
 // three-input max, then a tree.
@@ -247,6 +268,18 @@ struct AttendParams {
   // per-head factors of the stored keys and values (FP8 buffers), or null
   const float* k_scale;
   const float* v_scale;
+  // shared-O launches (d = 128 with a handle): one int per (query tile, head)
+  // item, set to 1 when a row's max left the fixed reference's headroom; the
+  // redo launch recomputes those items exactly and clears the flags
+  int* redo_flags;
+};
+
+// What the redo launch reads besides the attention's parameters: the raw
+// query and key/value segments.
+struct RedoInputs {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k[MAX_SEGS];
+  const __nv_bfloat16* v[MAX_SEGS];
 };
 
 // Segment and row of key tile j, and how many of its 128 rows are keys.
@@ -273,9 +306,8 @@ __device__ __forceinline__ void record_timeout(int* status) {
 // issues).  Descriptors are built once; the start-address field (bits 0-13,
 // in 16-byte units) is advanced by compile-time offsets, so the issuing warp
 // spends its cycles on tcgen05.mma and not on descriptor math.
-template <int D>
+template <int D, typename C>
 __device__ __forceinline__ void issue_s_warp(uint64_t dq, uint64_t dk, uint32_t d_s) {
-  using C = Cfg<D>;
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
     const uint64_t off = uint64_t(((kk / 4) * C::SUB_BYTES + (kk % 4) * 32) >> 4);
@@ -283,10 +315,9 @@ __device__ __forceinline__ void issue_s_warp(uint64_t dq, uint64_t dk, uint32_t 
   }
 }
 
-template <int D>
+template <int D, typename C>
 __device__ __forceinline__ void issue_pv_warp(uint64_t dv, uint32_t p_tmem, uint32_t d_o,
                                               uint32_t accumulate) {
-  using C = Cfg<D>;
 #pragma unroll
   for (int kk = 0; kk < BN / 16; ++kk)
     mma_ts_elect(d_o, p_tmem + kk * 8, dv + uint64_t((kk * 2048) >> 4), C::IDESC_O,
@@ -295,10 +326,11 @@ __device__ __forceinline__ void issue_pv_warp(uint64_t dv, uint32_t p_tmem, uint
 
 // SPLIT: the launch splits its last wave's query tiles by key range (see
 // AttendParams); a launch without a split uses the instantiation that has no
-// trace of it.
-template <int D, bool SPLIT>
+// trace of it.  SHARED (d = 128): the two warpgroups accumulate into one O
+// with one fixed exponent reference per row (Cfg::SHARED_O).
+template <int D, bool SPLIT, bool SHARED>
 __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_constant__ AttendParams p) {
-  using C = Cfg<D>;
+  using C = Cfg<D, SHARED>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -306,8 +338,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
   auto bar = [&](int i) -> uint32_t { return sbase + C::BAR_OFF + 8 * i; };
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  volatile int* overflow_flag = reinterpret_cast<volatile int*>(misc + 2);
   float* xch_m = reinterpret_cast<float*>(smem + C::XCH_OFF);
   float* xch_l = xch_m + 2 * BM;
+  float* xch0 = reinterpret_cast<float*>(smem + C::XCH0_OFF);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -354,7 +388,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
     for (int i = 0; i < 3; ++i) mbar_init(bar(C::B_DRAIN + i), 1);
     mbar_init(bar(C::B_COPY), 1);
     mbar_init(bar(C::B_COPY + 1), 1);
+    if (C::SHARED_O) mbar_init(bar(C::B_OFIRST), 1);
     misc[1] = 0;
+    if (C::SHARED_O) misc[2] = 0;
     fence_mbar_init();
   }
   if (warp == 9) {
@@ -503,7 +539,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
                                                            p.wait_limit)))
               return false;
             tc_fence_after();
-            issue_s_warp<D>(dq, dk0 + k_st * TILE16, tmem + (g ? C::S_COL1 : C::S_COL0));
+            issue_s_warp<D, C>(dq, dk0 + k_st * TILE16, tmem + (g ? C::S_COL1 : C::S_COL0));
             tc_commit_elect(bar(C::B_SFULL + g));
             tc_commit_elect(bar(C::B_KEMPTY + k_st));
             if (++k_st == C::NK) { k_st = 0; k_ph ^= 1; }
@@ -522,7 +558,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
             }
             pf_ph ^= 1u << g;
             tc_fence_after();
-            issue_pv_warp<D>(dv0 + v_st * TILE16, tmem + (g ? C::P_COL1 : C::P_COL0),
+            issue_pv_warp<D, C>(dv0 + v_st * TILE16, tmem + (g ? C::P_COL1 : C::P_COL0),
                              tmem + (g ? C::O_COL1 : C::O_COL0), j >= 2 ? 1u : 0u);
             tc_commit_elect(bar(C::B_ODONE + g));
             tc_commit_elect(bar(C::B_VEMPTY + v_st));
@@ -561,7 +597,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
             break;
           }
           tc_fence_after();
-          issue_s_warp<D>(dq, dk0 + k_st * TILE16, tmem + (g ? C::S_COL1 : C::S_COL0));
+          issue_s_warp<D, C>(dq, dk0 + k_st * TILE16, tmem + (g ? C::S_COL1 : C::S_COL0));
           tc_commit_elect(bar(C::B_SFULL + g));
           tc_commit_elect(bar(C::B_KEMPTY + k_st));
           if (++k_st == C::NK) { k_st = 0; k_ph ^= 1; }
@@ -585,10 +621,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
             break;
           }
           pf_ph ^= 1;
+          if (C::SHARED_O && j == 1 &&
+              !__all_sync(0xffffffffu, mbar_wait_bounded(bar(C::B_OFIRST), 0, abort_flag,
+                                                         p.wait_limit))) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
-          issue_pv_warp<D>(dv0 + v_st * TILE16, p_tm, o_tm, j >= 2 ? 1u : 0u);
+          issue_pv_warp<D, C>(dv0 + v_st * TILE16, p_tm, o_tm,
+                           (C::SHARED_O ? j >= 1 : j >= 2) ? 1u : 0u);
           tc_commit_elect(bar(C::B_ODONE + g));
           tc_commit_elect(bar(C::B_VEMPTY + v_st));
+          if (C::SHARED_O && j == 0) tc_commit_elect(bar(C::B_OFIRST));
         }
         if (ok) tc_commit_elect(bar(C::B_OFINAL));
       }
@@ -617,10 +661,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
     float l_run = 0.f;
     bool ok = true;
     int n = 0;
+    if (C::SHARED_O && wg >= nkv) {
+      // no tile for this warpgroup: take part in the reference exchange only
+      xch0[wg * BM + row] = -INFINITY;
+      named_bar_sync(2, 256);
+      m_ref = fmaxf(xch0[row], xch0[BM + row]);
+    }
     for (int j = wg; j < nkv; j += 2, ++n) {
       ok = mbar_wait_bounded(bar(C::B_SFULL + wg), n & 1, abort_flag, p.wait_limit);
       ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
+      if (!ok) {
+        if (C::SHARED_O && n == 0) {
+          xch0[wg * BM + row] = -INFINITY;
+          named_bar_sync(2, 256);
+        }
+        break;
+      }
       tc_fence_after();
       uint32_t sr[128];
       tmem_ld32_at<0>(s_addr, sr);
@@ -649,15 +705,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
       const float m_tile = row_max(s) * sl2;
       float alpha = 1.f;
       bool grow = false;
-      if (n == 0) {
-        m_ref = m_tile;
-      } else if (m_tile > m_ref + RESCALE_THRESHOLD) {
-        alpha = ex2_approx(m_ref - m_tile);
-        m_ref = m_tile;
-        grow = true;
+      float m_use;
+      if constexpr (C::SHARED_O) {
+        // one reference per row for both warpgroups: the larger of their first
+        // tiles' maxima, fixed from then on (no rescaling of the shared O)
+        if (n == 0) {
+          xch0[wg * BM + row] = m_tile;
+          named_bar_sync(2, 256);
+          m_ref = fmaxf(xch0[row], xch0[BM + row]);
+        }
+        m_use = fmaxf(m_ref, m_tile - SHARED_REF_HEADROOM);
+        if (m_use != m_ref) *overflow_flag = 1;
+      } else {
+        if (n == 0) {
+          m_ref = m_tile;
+        } else if (m_tile > m_ref + RESCALE_THRESHOLD) {
+          alpha = ex2_approx(m_ref - m_tile);
+          m_ref = m_tile;
+          grow = true;
+        }
+        m_use = m_ref;
       }
       uint32_t pk[64];
-      const float tile_sum = exp_tile<poly_pairs_per_8<D>()>(s, sl2, m_ref, pk);
+      const float tile_sum = exp_tile<poly_pairs_per_8<D>()>(s, sl2, m_use, pk);
       // l is rescaled by alpha (1 unless the reference grew) before this tile's sum
       l_run = l_run * alpha + tile_sum;
       if (n > 0) {
@@ -709,7 +779,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
       const float mf = fmaxf(m0, m1);
       const float a0 = ex2_approx(m0 - mf);
       const float a1 = nkv > 1 ? ex2_approx(m1 - mf) : 0.f;
-      const bool has1 = nkv > 1;
+      const bool has1 = !C::SHARED_O && nkv > 1;
       float* part = p.part + (cta - p.full_ctas) * int64_t(BM * (D + 2));
       const uint32_t o0 = tmem + lane_off + C::O_COL0;
       const uint32_t o1 = tmem + lane_off + C::O_COL1;
@@ -744,7 +814,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
       const float a1 = ex2_approx(m1 - mf);
       const float inv = (p.v_scale ? p.v_scale[head] : 1.f) / (l0 * a0 + l1 * a1);
       const float c0 = a0 * inv, c1 = a1 * inv;
-      const bool has1 = nkv > 1;
+      const bool has1 = !C::SHARED_O && nkv > 1;
       const int64_t qrow = int64_t(q_tile) * BM + row;
       __nv_bfloat16* orow = p.o + (qrow * p.heads + head) * D;
       const uint32_t o0 = tmem + lane_off + C::O_COL0;
@@ -781,6 +851,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0 && *abort_flag) record_timeout(p.status);
+  if (C::SHARED_O && threadIdx.x == 0 && *overflow_flag && p.redo_flags)
+    p.redo_flags[int64_t(head) * p.q_tiles + q_tile] = 1;
   if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
@@ -851,6 +923,72 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
+// Exact recomputation of the (query tile, head) items a shared-O launch
+// flagged (a row whose max outgrew the fixed reference's headroom): fp32
+// online softmax, one row at a time, over every key of every segment (the
+// same keys, scales and output as the attention launch), exp2f for the
+// exponentials.  Single-warp CTAs, one per SM, walk the items; an unflagged
+// item costs a load, a flagged item's flag is cleared.  Rare by
+// construction, so written for clarity, not speed.  One warp and at most 32
+// registers a thread make 1,024 registers, what an attention CTA (384 x 168)
+// leaves free on an SM, so a redo CTA can sit beside the next attention
+// launch's CTAs instead of holding them off.
+constexpr int REDO_THREADS = 32;
+template <int D>
+__global__ void __maxnreg__(32) redo_kernel(const __grid_constant__ AttendParams p,
+                                            const __grid_constant__ RedoInputs in) {
+  pdl_launch_dependents();
+  pdl_wait_prior();
+  const int64_t items = int64_t(p.q_tiles) * p.heads;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  constexpr int PER = D / 32;  // elements of a row per lane
+  for (int64_t item = blockIdx.x; item < items; item += gridDim.x) {
+    if (p.redo_flags[item] == 0) continue;
+    const int q_tile = static_cast<int>(item % p.q_tiles);
+    const int head = static_cast<int>(item / p.q_tiles);
+    const float sl2 = p.k_scale ? p.scale_log2 * p.k_scale[head] : p.scale_log2;
+    const float vs = p.v_scale ? p.v_scale[head] : 1.f;
+    for (int r = warp; r < BM; r += REDO_THREADS / 32) {
+      const int64_t qrow = int64_t(q_tile) * BM + r;
+      if (qrow >= p.lq) break;
+      float q[PER], o[PER];
+      const __nv_bfloat16* qp = in.q + (qrow * p.heads + head) * D + lane * PER;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        q[i] = __bfloat162float(qp[i]);
+        o[i] = 0.f;
+      }
+      float m = -INFINITY, l = 0.f;
+      for (int sg = 0; sg < p.nseg; ++sg) {
+        for (int64_t j = 0; j < p.seg_rows[sg]; ++j) {
+          const int64_t off = (j * p.heads + head) * D + lane * PER;
+          const __nv_bfloat16* kp = in.k[sg] + off;
+          float dot = 0.f;
+#pragma unroll
+          for (int i = 0; i < PER; ++i) dot = fmaf(q[i], __bfloat162float(kp[i]), dot);
+#pragma unroll
+          for (int w = 16; w >= 1; w /= 2) dot += __shfl_xor_sync(0xffffffffu, dot, w);
+          const float x = dot * sl2;
+          const float m_new = fmaxf(m, x);
+          const float corr = exp2f(m - m_new);
+          const float pj = exp2f(x - m_new);
+          l = l * corr + pj;
+          const __nv_bfloat16* vp = in.v[sg] + off;
+#pragma unroll
+          for (int i = 0; i < PER; ++i) o[i] = fmaf(pj, __bfloat162float(vp[i]), o[i] * corr);
+          m = m_new;
+        }
+      }
+      const float inv = vs / l;
+      __nv_bfloat16* op = p.o + (qrow * p.heads + head) * D + lane * PER;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) op[i] = __float2bfloat16_rn(o[i] * inv);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) p.redo_flags[item] = 0;
+  }
+}
+
 // [rows, heads, d] bf16, box = 128 rows x 1 head x 64 columns, 128-byte swizzle.
 bool encode_rows_map(CUtensorMap* m, const void* base, int64_t rows, int heads, int d) {
   auto enc = get_encode_fn();
@@ -871,9 +1009,10 @@ constexpr int MAX_DEVICES = 64;
 // for each instantiation.  setmaxnreg.inc waits until registers are free, so
 // the launch must carry exactly the budget the register split assumes, or the
 // kernel is not launched.
-template <int D>
-cudaError_t launch_d(const AttendParams& prm, dim3 grid, cudaStream_t stream) {
-  using C = Cfg<D>;
+template <int D, bool SHARED>
+cudaError_t launch_d(const AttendParams& prm, const RedoInputs& redo, dim3 grid,
+                     cudaStream_t stream) {
+  using C = Cfg<D, SHARED>;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES)
     return cudaErrorInvalidDevice;
@@ -892,10 +1031,13 @@ cudaError_t launch_d(const AttendParams& prm, dim3 grid, cudaStream_t stream) {
     });
     return attr_err[which][dev];
   };
-  cudaError_t e = split ? prepare(attend_kernel<D, true>, 1) : prepare(attend_kernel<D, false>, 0);
+  cudaError_t e = split ? prepare(attend_kernel<D, true, SHARED>, 1)
+                        : prepare(attend_kernel<D, false, SHARED>, 0);
   if (e != cudaSuccess) return e;
-  e = split ? launch_pdl(attend_kernel<D, true>, grid, dim3(NUM_THREADS), C::SMEM_ALLOC, stream, prm)
-            : launch_pdl(attend_kernel<D, false>, grid, dim3(NUM_THREADS), C::SMEM_ALLOC, stream, prm);
+  e = split ? launch_pdl(attend_kernel<D, true, SHARED>, grid, dim3(NUM_THREADS), C::SMEM_ALLOC,
+                         stream, prm)
+            : launch_pdl(attend_kernel<D, false, SHARED>, grid, dim3(NUM_THREADS), C::SMEM_ALLOC,
+                         stream, prm);
   if (e == cudaSuccess && split)
     e = launch_pdl(combine_kernel<D>,
                    dim3(static_cast<unsigned>(split_tiles),
@@ -903,6 +1045,12 @@ cudaError_t launch_d(const AttendParams& prm, dim3 grid, cudaStream_t stream) {
                    dim3(COMBINE_THREADS), 0, stream,
                    static_cast<const float*>(prm.part), prm.full_ctas, prm.q_tiles, prm.split_chunks,
                    prm.lq, prm.heads, prm.v_scale, prm.o);
+  if constexpr (SHARED)
+    if (e == cudaSuccess)
+      e = launch_pdl(redo_kernel<D>,
+                     dim3(static_cast<unsigned>(std::min<int64_t>(int64_t(prm.q_tiles) * prm.heads,
+                                                                  device_sm_count()))),
+                     dim3(REDO_THREADS), 0, stream, prm, redo);
   return e;
 }
 
@@ -913,9 +1061,11 @@ bool attend_copies_in_kernel(int d) { return Cfg<64>::COPY_IN_KERNEL && d == 64;
 cudaError_t launch_attend(const void* q, void* o, int64_t lq, const KVSegment* segs, int nseg,
                           int heads, int d, int* status, const RecordCopy* copy,
                           unsigned long long wait_limit, const float* k_scale,
-                          const float* v_scale, float* part, int part_ctas, cudaStream_t stream) {
+                          const float* v_scale, float* part, int part_ctas, int* redo_flags,
+                          cudaStream_t stream) {
   if (nseg < 1 || nseg > MAX_SEGS) return cudaErrorInvalidValue;
   AttendParams prm = {};
+  RedoInputs redo = {};
   if (!encode_rows_map(&prm.tm_q, q, lq, heads, d)) return cudaErrorInvalidValue;
   int tiles = 0;
   for (int k = 0; k < nseg; ++k) {
@@ -926,8 +1076,11 @@ cudaError_t launch_attend(const void* q, void* o, int64_t lq, const KVSegment* s
     tiles += static_cast<int>((segs[k].rows + BN - 1) / BN);
     prm.seg_tiles_end[k] = tiles;
     prm.seg_rows[k] = static_cast<int>(segs[k].rows);
+    redo.k[k] = static_cast<const __nv_bfloat16*>(segs[k].k);
+    redo.v[k] = static_cast<const __nv_bfloat16*>(segs[k].v);
   }
   prm.nseg = nseg;
+  redo.q = static_cast<const __nv_bfloat16*>(q);
   prm.o = static_cast<__nv_bfloat16*>(o);
   prm.lq = lq;
   prm.heads = heads;
@@ -972,8 +1125,14 @@ cudaError_t launch_attend(const void* q, void* o, int64_t lq, const KVSegment* s
       }
     }
   }
-  if (d == 64) return launch_d<64>(prm, grid, stream);
-  if (d == 128) return launch_d<128>(prm, grid, stream);
+  if (d == 64) return launch_d<64, false>(prm, redo, grid, stream);
+  if (d == 128 && redo_flags) {
+    // one O for both warpgroups, fixed exponent references, exact redo of
+    // flagged items (needs the caller's per-item flag array)
+    prm.redo_flags = redo_flags;
+    return launch_d<128, true>(prm, redo, grid, stream);
+  }
+  if (d == 128) return launch_d<128, false>(prm, redo, grid, stream);
   return cudaErrorInvalidValue;
 }
 
