@@ -82,16 +82,9 @@ enum {
  * The handle also holds a scratch of (SM count) * 128 * (d + 2) floats: an
  * attention launch of more than one wave of (query tile, head) CTAs whose
  * last wave is at most half full splits that wave's query tiles by key range
- * and merges the partial results in a second launch.  With d = 128 the handle
- * also holds one int per (query tile, head) of its attention calls,
- * ceil(R / 128) * heads: its attention launches share one output accumulator
- * between their two softmax warpgroups, with each row's exponent reference
- * fixed from their first key tiles, and flag there any item whose row max
- * later exceeds that reference by more than 2^64; a follow-up launch
- * recomputes the flagged items exactly (in fp32) and clears the flags.
- * Attention calls on one handle whose launches can overlap on the device
- * (different streams with no event between them) may share this state and
- * must be ordered.
+ * and merges the partial results in a second launch.  Attention calls on one
+ * handle whose launches can overlap on the device (different streams with no
+ * event between them) may share that scratch and must be ordered.
  * Requirements: blocks >= 1, heads >= 1, d in {64, 128}, grid_h >= 1,
  * grid_w >= 1, X >= 1, 0 <= Y <= W (W == Y gives an empty SUM region).
  * Returns WM_ERR_INVALID_ARG / WM_ERR_UNSUPPORTED before touching the device,

@@ -14,8 +14,7 @@
 //   warps 10/11 issue O_g += P_j V_j for even / odd tiles (tcgen05.mma TS: P
 //               from TMEM, V MN-major in smem); three issuing warps keep the
 //               tensor core fed while each waits on barriers and commits.
-//               d = 128 without a redo-flag array: warp 9 issues everything,
-//               in order.
+//               (the same for d = 128, whose two warpgroups share one O).
 //   warps 0-3   softmax warpgroup 0: even key tiles, S0/P0/O0 in TMEM
 //   warps 4-7   softmax warpgroup 1: odd key tiles, S1/P1/O1 in TMEM
 // The control warpgroup gives registers back (setmaxnreg) so that each
@@ -32,18 +31,15 @@
 //   of tile j-2 finished: O_g is stable and P_g is free; waiting only now
 //   hides the MMA round trip behind the exponentials) -> rescale O_g if m
 //   moved -> P as bf16 into TMEM -> arrive P_full[g].
-// d = 128 has two layouts.  Shared O (attention calls of a handle, which
-// owns a per-item flag array): the two warpgroups attend for the same rows,
-// so both P.V issuers accumulate into one O (2 S + 2 P + 1 O of 128, 64,
-// 128 columns), and each row's exponent reference is fixed from the larger
-// of the two warpgroups' first-tile maxima (exchanged once) instead of moved
-// lazily -- S is then released as soon as it is read, as for d = 64.  A tile
-// whose row max exceeds that reference by more than 2^64 (the fp32 headroom
-// of the accumulation) is computed against a clamped reference and its item
-// flagged; a redo launch recomputes flagged items exactly.  Per-warpgroup O
-// (dense calls, no flag array): the TMEM budget (2 S + 2 O of 128 columns)
-// leaves no room for a separate P, so P overwrites the first half of S and
-// S_{j+2} is issued only after P_j.V_j has completed (O_done).
+// For d = 128 the two warpgroups, which attend for the same rows, share one
+// O: both P.V issuers accumulate into it (2 S + 2 P + 1 O of 128, 64, 128
+// columns), so P has columns of its own and S is released as soon as it is
+// read, as for d = 64.  A shared O cannot be rescaled lazily, so each row's
+// exponent reference is fixed: the larger of the two warpgroups' first-tile
+// maxima, exchanged once.  A tile whose row max exceeds it by more than 2^64
+// (the fp32 headroom of the accumulation) is computed against a clamped
+// reference and the CTA flagged; before it exits, a flagged CTA recomputes
+// its rows exactly in fp32 and overwrites what its epilogue wrote.
 // The two warpgroups' partial results (m, l, O) are merged row by row at the
 // end and stored as bf16.
 //
@@ -268,18 +264,12 @@ struct AttendParams {
   // per-head factors of the stored keys and values (FP8 buffers), or null
   const float* k_scale;
   const float* v_scale;
-  // shared-O launches (d = 128 with a handle): one int per (query tile, head)
-  // item, set to 1 when a row's max left the fixed reference's headroom; the
-  // redo launch recomputes those items exactly and clears the flags
-  int* redo_flags;
-};
-
-// What the redo launch reads besides the attention's parameters: the raw
-// query and key/value segments.
-struct RedoInputs {
+  // the raw query and key/value segments, read only by the exact
+  // recomputation of a shared-O CTA whose row maxima outgrew the fixed
+  // references (d = 128)
   const __nv_bfloat16* q;
-  const __nv_bfloat16* k[MAX_SEGS];
-  const __nv_bfloat16* v[MAX_SEGS];
+  const __nv_bfloat16* seg_k[MAX_SEGS];
+  const __nv_bfloat16* seg_v[MAX_SEGS];
 };
 
 // Segment and row of key tile j, and how many of its 128 rows are keys.
@@ -322,6 +312,69 @@ __device__ __forceinline__ void issue_pv_warp(uint64_t dv, uint32_t p_tmem, uint
   for (int kk = 0; kk < BN / 16; ++kk)
     mma_ts_elect(d_o, p_tmem + kk * 8, dv + uint64_t((kk * 2048) >> 4), C::IDESC_O,
                  (accumulate | uint32_t(kk > 0)));
+}
+
+// Exact recomputation of a shared-O CTA's rows when one of its tiles had a
+// row max beyond the fixed reference's headroom: fp32 online softmax, one row
+// per warp at a time (all twelve warps), over the CTA's own key tiles, read
+// straight from the segments; exp2f for the exponentials.  Writes what the
+// epilogue wrote: the bf16 output rows, or for a key-range piece its
+// unnormalised partial O, reference and sum.  Rare by construction, so
+// written for clarity, not speed.
+template <int D>
+__device__ void exact_rows(const AttendParams& p, int q_tile, int head, int j0, int nkv,
+                           float* part) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  constexpr int NW = NUM_THREADS / 32;
+  constexpr int PER = D / 32;  // elements of a row per lane
+  const float sl2 = p.k_scale ? p.scale_log2 * p.k_scale[head] : p.scale_log2;
+  const float vs = p.v_scale ? p.v_scale[head] : 1.f;
+  for (int r = warp; r < BM; r += NW) {
+    const int64_t qrow = int64_t(q_tile) * BM + r;
+    if (qrow >= p.lq) break;
+    float q[PER], o[PER];
+    const __nv_bfloat16* qp = p.q + (qrow * p.heads + head) * D + lane * PER;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      q[i] = __bfloat162float(qp[i]);
+      o[i] = 0.f;
+    }
+    float m = -INFINITY, l = 0.f;
+    for (int t = 0; t < nkv; ++t) {
+      const TileLoc tl = tile_loc(p, j0 + t);
+      const __nv_bfloat16* kb = p.seg_k[tl.seg];
+      const __nv_bfloat16* vb = p.seg_v[tl.seg];
+      for (int jj = 0; jj < tl.valid; ++jj) {
+        const int64_t off = ((int64_t(tl.row) + jj) * p.heads + head) * D + lane * PER;
+        float dot = 0.f;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) dot = fmaf(q[i], __bfloat162float(kb[off + i]), dot);
+#pragma unroll
+        for (int w = 16; w >= 1; w /= 2) dot += __shfl_xor_sync(0xffffffffu, dot, w);
+        const float x = dot * sl2;
+        const float m_new = fmaxf(m, x);
+        const float corr = exp2f(m - m_new);
+        const float pj = exp2f(x - m_new);
+        l = l * corr + pj;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) o[i] = fmaf(pj, __bfloat162float(vb[off + i]), o[i] * corr);
+        m = m_new;
+      }
+    }
+    if (part) {
+#pragma unroll
+      for (int i = 0; i < PER; ++i) part[r * D + lane * PER + i] = o[i];
+      if (lane == 0) {
+        part[BM * D + r] = m;
+        part[BM * D + BM + r] = l;
+      }
+    } else {
+      const float inv = vs / l;
+      __nv_bfloat16* op = p.o + (qrow * p.heads + head) * D + lane * PER;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) op[i] = __float2bfloat16_rn(o[i] * inv);
+    }
+  }
 }
 
 // SPLIT: the launch splits its last wave's query tiles by key range (see
@@ -851,8 +904,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_kernel(const __grid_con
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0 && *abort_flag) record_timeout(p.status);
-  if (C::SHARED_O && threadIdx.x == 0 && *overflow_flag && p.redo_flags)
-    p.redo_flags[int64_t(head) * p.q_tiles + q_tile] = 1;
+  if constexpr (C::SHARED_O) {
+    if (*overflow_flag && !*abort_flag)
+      exact_rows<D>(p, q_tile, head, j0, nkv,
+                    split ? p.part + (cta - p.full_ctas) * int64_t(BM * (D + 2)) : nullptr);
+  }
   if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
@@ -923,72 +979,6 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
-// Exact recomputation of the (query tile, head) items a shared-O launch
-// flagged (a row whose max outgrew the fixed reference's headroom): fp32
-// online softmax, one row at a time, over every key of every segment (the
-// same keys, scales and output as the attention launch), exp2f for the
-// exponentials.  Single-warp CTAs, one per SM, walk the items; an unflagged
-// item costs a load, a flagged item's flag is cleared.  Rare by
-// construction, so written for clarity, not speed.  One warp and at most 32
-// registers a thread make 1,024 registers, what an attention CTA (384 x 168)
-// leaves free on an SM, so a redo CTA can sit beside the next attention
-// launch's CTAs instead of holding them off.
-constexpr int REDO_THREADS = 32;
-template <int D>
-__global__ void __maxnreg__(32) redo_kernel(const __grid_constant__ AttendParams p,
-                                            const __grid_constant__ RedoInputs in) {
-  pdl_launch_dependents();
-  pdl_wait_prior();
-  const int64_t items = int64_t(p.q_tiles) * p.heads;
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  constexpr int PER = D / 32;  // elements of a row per lane
-  for (int64_t item = blockIdx.x; item < items; item += gridDim.x) {
-    if (p.redo_flags[item] == 0) continue;
-    const int q_tile = static_cast<int>(item % p.q_tiles);
-    const int head = static_cast<int>(item / p.q_tiles);
-    const float sl2 = p.k_scale ? p.scale_log2 * p.k_scale[head] : p.scale_log2;
-    const float vs = p.v_scale ? p.v_scale[head] : 1.f;
-    for (int r = warp; r < BM; r += REDO_THREADS / 32) {
-      const int64_t qrow = int64_t(q_tile) * BM + r;
-      if (qrow >= p.lq) break;
-      float q[PER], o[PER];
-      const __nv_bfloat16* qp = in.q + (qrow * p.heads + head) * D + lane * PER;
-#pragma unroll
-      for (int i = 0; i < PER; ++i) {
-        q[i] = __bfloat162float(qp[i]);
-        o[i] = 0.f;
-      }
-      float m = -INFINITY, l = 0.f;
-      for (int sg = 0; sg < p.nseg; ++sg) {
-        for (int64_t j = 0; j < p.seg_rows[sg]; ++j) {
-          const int64_t off = (j * p.heads + head) * D + lane * PER;
-          const __nv_bfloat16* kp = in.k[sg] + off;
-          float dot = 0.f;
-#pragma unroll
-          for (int i = 0; i < PER; ++i) dot = fmaf(q[i], __bfloat162float(kp[i]), dot);
-#pragma unroll
-          for (int w = 16; w >= 1; w /= 2) dot += __shfl_xor_sync(0xffffffffu, dot, w);
-          const float x = dot * sl2;
-          const float m_new = fmaxf(m, x);
-          const float corr = exp2f(m - m_new);
-          const float pj = exp2f(x - m_new);
-          l = l * corr + pj;
-          const __nv_bfloat16* vp = in.v[sg] + off;
-#pragma unroll
-          for (int i = 0; i < PER; ++i) o[i] = fmaf(pj, __bfloat162float(vp[i]), o[i] * corr);
-          m = m_new;
-        }
-      }
-      const float inv = vs / l;
-      __nv_bfloat16* op = p.o + (qrow * p.heads + head) * D + lane * PER;
-#pragma unroll
-      for (int i = 0; i < PER; ++i) op[i] = __float2bfloat16_rn(o[i] * inv);
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) p.redo_flags[item] = 0;
-  }
-}
-
 // [rows, heads, d] bf16, box = 128 rows x 1 head x 64 columns, 128-byte swizzle.
 bool encode_rows_map(CUtensorMap* m, const void* base, int64_t rows, int heads, int d) {
   auto enc = get_encode_fn();
@@ -1010,8 +1000,7 @@ constexpr int MAX_DEVICES = 64;
 // the launch must carry exactly the budget the register split assumes, or the
 // kernel is not launched.
 template <int D, bool SHARED>
-cudaError_t launch_d(const AttendParams& prm, const RedoInputs& redo, dim3 grid,
-                     cudaStream_t stream) {
+cudaError_t launch_d(const AttendParams& prm, dim3 grid, cudaStream_t stream) {
   using C = Cfg<D, SHARED>;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES)
@@ -1045,12 +1034,6 @@ cudaError_t launch_d(const AttendParams& prm, const RedoInputs& redo, dim3 grid,
                    dim3(COMBINE_THREADS), 0, stream,
                    static_cast<const float*>(prm.part), prm.full_ctas, prm.q_tiles, prm.split_chunks,
                    prm.lq, prm.heads, prm.v_scale, prm.o);
-  if constexpr (SHARED)
-    if (e == cudaSuccess)
-      e = launch_pdl(redo_kernel<D>,
-                     dim3(static_cast<unsigned>(std::min<int64_t>(int64_t(prm.q_tiles) * prm.heads,
-                                                                  device_sm_count()))),
-                     dim3(REDO_THREADS), 0, stream, prm, redo);
   return e;
 }
 
@@ -1061,11 +1044,9 @@ bool attend_copies_in_kernel(int d) { return Cfg<64>::COPY_IN_KERNEL && d == 64;
 cudaError_t launch_attend(const void* q, void* o, int64_t lq, const KVSegment* segs, int nseg,
                           int heads, int d, int* status, const RecordCopy* copy,
                           unsigned long long wait_limit, const float* k_scale,
-                          const float* v_scale, float* part, int part_ctas, int* redo_flags,
-                          cudaStream_t stream) {
+                          const float* v_scale, float* part, int part_ctas, cudaStream_t stream) {
   if (nseg < 1 || nseg > MAX_SEGS) return cudaErrorInvalidValue;
   AttendParams prm = {};
-  RedoInputs redo = {};
   if (!encode_rows_map(&prm.tm_q, q, lq, heads, d)) return cudaErrorInvalidValue;
   int tiles = 0;
   for (int k = 0; k < nseg; ++k) {
@@ -1076,11 +1057,11 @@ cudaError_t launch_attend(const void* q, void* o, int64_t lq, const KVSegment* s
     tiles += static_cast<int>((segs[k].rows + BN - 1) / BN);
     prm.seg_tiles_end[k] = tiles;
     prm.seg_rows[k] = static_cast<int>(segs[k].rows);
-    redo.k[k] = static_cast<const __nv_bfloat16*>(segs[k].k);
-    redo.v[k] = static_cast<const __nv_bfloat16*>(segs[k].v);
+    prm.seg_k[k] = static_cast<const __nv_bfloat16*>(segs[k].k);
+    prm.seg_v[k] = static_cast<const __nv_bfloat16*>(segs[k].v);
   }
   prm.nseg = nseg;
-  redo.q = static_cast<const __nv_bfloat16*>(q);
+  prm.q = static_cast<const __nv_bfloat16*>(q);
   prm.o = static_cast<__nv_bfloat16*>(o);
   prm.lq = lq;
   prm.heads = heads;
@@ -1125,14 +1106,8 @@ cudaError_t launch_attend(const void* q, void* o, int64_t lq, const KVSegment* s
       }
     }
   }
-  if (d == 64) return launch_d<64, false>(prm, redo, grid, stream);
-  if (d == 128 && redo_flags) {
-    // one O for both warpgroups, fixed exponent references, exact redo of
-    // flagged items (needs the caller's per-item flag array)
-    prm.redo_flags = redo_flags;
-    return launch_d<128, true>(prm, redo, grid, stream);
-  }
-  if (d == 128) return launch_d<128, false>(prm, redo, grid, stream);
+  if (d == 64) return launch_d<64, false>(prm, grid, stream);
+  if (d == 128) return launch_d<128, true>(prm, grid, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -48,10 +48,6 @@ struct wm_kvbuf {
   // by key range: part_ctas x 128 x (d + 2) floats (part_ctas = SM count)
   float* part = nullptr;
   int part_ctas = 0;
-  // head dimension 128: one int per (query tile, head) of an attention call
-  // (ceil(R / 128) x heads), the items a shared-O launch flagged for an exact
-  // recomputation (zero between calls)
-  int* redo = nullptr;
 };
 
 namespace {
@@ -162,7 +158,6 @@ static int kvbuf_create(wm_kvbuf** out, int blocks, int heads, int d, int grid_h
     cudaFree(h->scales);
     cudaFree(h->widened);
     cudaFree(h->part);
-    cudaFree(h->redo);
     delete h;
     if (e == cudaErrorMemoryAllocation) {
       cudaGetLastError();
@@ -178,11 +173,7 @@ static int kvbuf_create(wm_kvbuf** out, int blocks, int heads, int d, int grid_h
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&h->part_ctas, cudaDevAttrMultiProcessorCount, h->device);
   if (e == cudaSuccess)
     e = cudaMalloc(&h->part, size_t(h->part_ctas) * 128 * (d + 2) * sizeof(float));
-  if (e == cudaSuccess && d == 128) {
-    const size_t items = size_t((h->R + 127) / 128) * size_t(heads);
-    e = cudaMalloc(&h->redo, items * sizeof(int));
-    if (e == cudaSuccess) e = cudaMemset(h->redo, 0, items * sizeof(int));
-  }
+
   if (e == cudaSuccess && kv_format == WM_KV_E4M3) {
     const size_t ns = size_t(blocks) * heads;
     e = cudaMalloc(&h->scales, 2 * ns * sizeof(float));
@@ -222,7 +213,6 @@ int wm_kvbuf_destroy(wm_kvbuf* h) {
   cudaFree(h->scales);
   cudaFree(h->widened);
   cudaFree(h->part);
-  cudaFree(h->redo);
   cudaSetDevice(dev);
   delete h;
   return e == cudaSuccess ? WM_OK : cuda_fail(e);
@@ -323,11 +313,11 @@ static cudaError_t attend_prefix(wm_kvbuf* h, int block, const void* Q, void* O,
     const wmkv::KVSegment seg = {wk, wv, end};
     return wmkv::launch_attend(Q, O, h->R, &seg, 1, h->heads, h->d, h->status, nullptr, h->wait_limit,
                                block_k_scale(h, block), block_v_scale(h, block), h->part,
-                               h->part_ctas, h->redo, s);
+                               h->part_ctas, s);
   }
   const wmkv::KVSegment seg = {kbuf, vbuf, end};
   return wmkv::launch_attend(Q, O, h->R, &seg, 1, h->heads, h->d, h->status, nullptr, h->wait_limit,
-                             nullptr, nullptr, h->part, h->part_ctas, h->redo, s);
+                             nullptr, nullptr, h->part, h->part_ctas, s);
 }
 
 int wm_write_record(wm_kvbuf* h, int block, int64_t t, const void* K, const void* V,
@@ -387,7 +377,7 @@ int wm_write_attend(wm_kvbuf* h, int block, int64_t t, const void* Q, const void
     if (e == cudaSuccess)
       e = wmkv::launch_attend(Q, O, h->R, &seg, 1, h->heads, h->d, h->status, nullptr, h->wait_limit,
                               block_k_scale(h, block), block_v_scale(h, block), h->part,
-                              h->part_ctas, h->redo, s);
+                              h->part_ctas, s);
   } else if (wmkv::attend_copies_in_kernel(h->d)) {
     // keys: buffer rows before the slot, buffer rows after it, and the record
     // itself from the caller (the slot is being written by the same launch)
@@ -400,13 +390,13 @@ int wm_write_attend(wm_kvbuf* h, int block, int64_t t, const void* Q, const void
     segs[nseg++] = {K, V, h->R};
     const wmkv::RecordCopy cp = {K, V, kslot, vslot, n16};
     e = wmkv::launch_attend(Q, O, h->R, segs, nseg, h->heads, h->d, h->status, &cp, h->wait_limit,
-                            nullptr, nullptr, h->part, h->part_ctas, h->redo, s);
+                            nullptr, nullptr, h->part, h->part_ctas, s);
   } else {
     e = wmkv::launch_copy_pair(K, V, kslot, vslot, n16, s);
     const wmkv::KVSegment seg = {kbuf, vbuf, end};
     if (e == cudaSuccess)
       e = wmkv::launch_attend(Q, O, h->R, &seg, 1, h->heads, h->d, h->status, nullptr,
-                              h->wait_limit, nullptr, nullptr, h->part, h->part_ctas, h->redo, s);
+                              h->wait_limit, nullptr, nullptr, h->part, h->part_ctas, s);
   }
   if (e != cudaSuccess) return cuda_fail(e);
   h->written[block] = t;
@@ -488,7 +478,7 @@ int wm_attend_dense(const void* Q, const void* K, const void* V, void* O, int64_
   const wmkv::KVSegment seg = {K, V, Lk};
   cudaError_t e = wmkv::launch_attend(Q, O, Lq, &seg, 1, heads, d, dev_status, nullptr,
                                       wmkv::DEFAULT_WAIT_LIMIT_CYCLES, nullptr, nullptr, nullptr, 0,
-                                      nullptr, reinterpret_cast<cudaStream_t>(stream));
+                                      reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
   return WM_OK;
 }
@@ -514,7 +504,7 @@ int wm_attend_dense_fp8(const void* Q, const void* K8, const void* V8, const flo
   const wmkv::KVSegment seg = {wk, wv, Lk};
   if (e == cudaSuccess)
     e = wmkv::launch_attend(Q, O, Lq, &seg, 1, heads, d, dev_status, nullptr,
-                            wmkv::DEFAULT_WAIT_LIMIT_CYCLES, k_scale, v_scale, nullptr, 0, nullptr, s);
+                            wmkv::DEFAULT_WAIT_LIMIT_CYCLES, k_scale, v_scale, nullptr, 0, s);
   if (e != cudaSuccess) return cuda_fail(e);
   return WM_OK;
 }

@@ -67,19 +67,10 @@ constexpr unsigned long long DEFAULT_WAIT_LIMIT_CYCLES = 4000000000ull;
 // lets a launch of more than one wave of CTAs split the query tiles of its
 // last, partial wave by key range (a second, combine launch follows); null
 // keeps one CTA per (query tile, head).
-//
-// redo_flags (device, ceil(lq / 128) x heads ints, zero-initialised, may be
-// null): with it, a head-dimension-128 launch uses the shared-O layout (one O
-// for both softmax warpgroups, one fixed exponent reference per row) and
-// flags the (query tile, head) items where a row's max outgrew that
-// reference's headroom; a third launch recomputes the flagged items exactly
-// and clears their flags.  Null keeps the per-warpgroup O with lazy
-// rescaling.  Calls sharing a flag array must be ordered on the device.
 cudaError_t launch_attend(const void* q, void* o, int64_t lq, const KVSegment* segs, int nseg,
                           int heads, int d, int* status, const RecordCopy* copy,
                           unsigned long long wait_limit, const float* k_scale,
-                          const float* v_scale, float* part, int part_ctas, int* redo_flags,
-                          cudaStream_t stream);
+                          const float* v_scale, float* part, int part_ctas, cudaStream_t stream);
 bool attend_copies_in_kernel(int d);
 
 // Keeps the CUDA error's text for wm_last_cuda_error; returns WM_ERR_CUDA.
